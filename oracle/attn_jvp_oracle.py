@@ -1,0 +1,174 @@
+"""Float64 CPU oracle for custom-mask attention and its Jacobian-vector product.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path may import this module:
+only tests, the smoke check and the benchmark's CPU-baseline leg use it. It
+shares no code with the CUDA library.
+
+What it computes (Causal-rCM summary page, App. B "FlashAttention-2 JVP Kernel
+with Custom Masks"): for every query row i, with admissible key set A(i) given
+by the mask predicate below,
+
+    S_ij  = s * (q_i . k_j)                              j in A(i)
+    LSE_i = log sum_{j in A(i)} exp(S_ij)                (natural log)
+    P_ij  = exp(S_ij - LSE_i),  P_ij = 0 for j not in A(i)
+    O_i   = sum_j P_ij v_j
+    tS_ij = s * (tq_i . k_j + q_i . tk_j)
+    mu_i  = sum_j P_ij tS_ij
+    tO_i  = sum_j P_ij (tS_ij - mu_i) v_j + sum_j P_ij tv_j
+
+This is the plain dense definition of O = softmax(S + M) V and of its
+directional derivative along (tq, tk, tv): the derivative of the softmax row
+is tP = P * (tS - rowsum(P * tS)), masked entries carry no tangent because the
+discrete mask has none (App. B), and tO = tP V + P tV. It is evaluated
+directly, not through the online-softmax recurrence the kernel uses.
+
+Mask (App. B; section 3 "Continuous-time consistency": the TF-masked packed
+forward; Causal Forcing summary page, section 2: clean and noisy videos
+concatenated under a causal attention mask). The sequence is
+[clean chunks | noisy chunks], n chunks of c tokens each, L = 2 n c:
+  * a clean query in chunk j sees clean keys in chunks <= j and no noisy key;
+  * a noisy query in chunk i sees clean keys in chunks < i and the noisy keys
+    of its own chunk i.
+Block-causal mode (Causal-rCM page, section 2 "Autoregressive video
+diffusion": causal over temporal blocks, full attention inside a block):
+L = n c and a query in chunk j sees keys in chunks <= j.
+Attention inside a chunk is full (bidirectional).
+
+Every function here is pinned by tests/test_oracle_pins.py against values
+that do not come from this file: finite differences, an autodiff JVP of the
+library softmax attention, hand-derived closed forms, hand-written masks,
+invariants and pair-count formulas.
+"""
+from __future__ import annotations
+
+import math
+from typing import Iterable, Optional, Sequence, Tuple
+
+import numpy as np
+
+TEACHER_FORCING = 0
+BLOCK_CAUSAL = 1
+
+
+def seq_len(mode: int, chunk_tokens: int, n_chunks: int) -> int:
+    """L = 2 n c for the packed teacher-forcing sequence, n c otherwise."""
+    return (2 if mode == TEACHER_FORCING else 1) * n_chunks * chunk_tokens
+
+
+def allowed(mode: int, c: int, n: int, i, j) -> np.ndarray:
+    """Mask predicate: True where query token i may attend to key token j.
+
+    `i` and `j` broadcast against each other (0-based token indices)."""
+    i = np.asarray(i, dtype=np.int64)
+    j = np.asarray(j, dtype=np.int64)
+    if mode == BLOCK_CAUSAL:
+        return (j // c) <= (i // c)
+    if mode != TEACHER_FORCING:
+        raise ValueError(f"unknown mask mode {mode}")
+    nc = n * c
+    i_clean = i < nc
+    j_clean = j < nc
+    ci = np.where(i_clean, i // c, (i - nc) // c)     # chunk of the query
+    cj = np.where(j_clean, j // c, (j - nc) // c)     # chunk of the key
+    clean_q = i_clean & j_clean & (cj <= ci)
+    noisy_q_clean_k = (~i_clean) & j_clean & (cj < ci)
+    noisy_q_noisy_k = (~i_clean) & (~j_clean) & (cj == ci)
+    return clean_q | noisy_q_clean_k | noisy_q_noisy_k
+
+
+def mask_matrix(mode: int, c: int, n: int) -> np.ndarray:
+    """Explicit [L, L] boolean mask (small L only)."""
+    L = seq_len(mode, c, n)
+    t = np.arange(L)
+    return allowed(mode, c, n, t[:, None], t[None, :])
+
+
+def count_pairs_bruteforce(mode: int, c: int, n: int) -> int:
+    """Number of admissible (query, key) pairs, counted from the predicate."""
+    L = seq_len(mode, c, n)
+    t = np.arange(L)
+    total = 0
+    for i0 in range(0, L, 4096):
+        rows = t[i0:i0 + 4096]
+        total += int(allowed(mode, c, n, rows[:, None], t[None, :]).sum())
+    return total
+
+
+def _as64(x) -> np.ndarray:
+    """Promote a tensor (numpy or torch, any float dtype) to float64 numpy,
+    bit-exactly for bf16/fp32 inputs."""
+    if hasattr(x, "detach"):  # torch tensor: bf16 has no numpy dtype
+        import torch
+        return x.detach().to("cpu", torch.float64).numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def attn_jvp_rows(q, k, v, tq, tk, tv, mode: int, c: int, n: int,
+                  scale: Optional[float], rows: Sequence[int],
+                  block: int = 64) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """O, tO and LSE for the given query rows of ONE (batch, head).
+
+    q..tv are [L, d] (any float type; promoted to float64). Returns
+    O [R, d], tO [R, d], LSE [R] in float64 for R = len(rows)."""
+    q, k, v, tq, tk, tv = (_as64(x) for x in (q, k, v, tq, tk, tv))
+    L, d = q.shape
+    s = (1.0 / math.sqrt(d)) if scale is None else float(scale)
+    rows = np.asarray(rows, dtype=np.int64)
+    R = rows.shape[0]
+    O = np.empty((R, d))
+    tO = np.empty((R, d))
+    lse = np.empty(R)
+    keys = np.arange(L)
+    for r0 in range(0, R, block):
+        rr = rows[r0:r0 + block]
+        M = allowed(mode, c, n, rr[:, None], keys[None, :])           # [r, L]
+        S = s * (q[rr] @ k.T)                                        # [r, L]
+        S = np.where(M, S, -np.inf)
+        smax = S.max(axis=1, keepdims=True)                          # finite: A(i) is never empty
+        lse_r = smax[:, 0] + np.log(np.exp(S - smax).sum(axis=1))
+        P = np.exp(S - lse_r[:, None])                               # 0 where masked
+        tS = s * (tq[rr] @ k.T + q[rr] @ tk.T)
+        tS = np.where(M, tS, 0.0)
+        mu = (P * tS).sum(axis=1, keepdims=True)
+        tP = P * (tS - mu)
+        O[r0:r0 + block] = P @ v
+        tO[r0:r0 + block] = tP @ v + P @ tv
+        lse[r0:r0 + block] = lse_r
+    return O, tO, lse
+
+
+def attn_jvp_dense(q, k, v, tq, tk, tv, mode: int, c: int, n: int,
+                   scale: Optional[float] = None):
+    """Full outputs for [B, L, H, d] inputs: O, tO [B, L, H, d] and LSE
+    [B, H, L], all float64 numpy."""
+    q, k, v, tq, tk, tv = (_as64(x) for x in (q, k, v, tq, tk, tv))
+    B, L, H, d = q.shape
+    if L != seq_len(mode, c, n):
+        raise ValueError("L does not match the mask (mode, chunk_tokens, n_chunks)")
+    O = np.empty((B, L, H, d))
+    tO = np.empty((B, L, H, d))
+    lse = np.empty((B, H, L))
+    allrows = np.arange(L)
+    for b in range(B):
+        for h in range(H):
+            o_, to_, l_ = attn_jvp_rows(q[b, :, h], k[b, :, h], v[b, :, h],
+                                        tq[b, :, h], tk[b, :, h], tv[b, :, h],
+                                        mode, c, n, scale, allrows)
+            O[b, :, h] = o_
+            tO[b, :, h] = to_
+            lse[b, h] = l_
+    return O, tO, lse
+
+
+def attn_forward_dense(q, k, v, mode: int, c: int, n: int,
+                       scale: Optional[float] = None):
+    """Primal output only (O and LSE); used to take finite differences."""
+    z = np.zeros_like(_as64(q))
+    O, _, lse = attn_jvp_dense(q, k, v, z, z, z, mode, c, n, scale)
+    return O, lse
+
+
+def effective_flops(pairs: int, d: int) -> int:
+    """Algorithmic FLOPs of one call: 12 d per admissible pair (S: 2d,
+    tS: 4d, P V: 2d, tP V + P tV: 4d)."""
+    return 12 * d * pairs

@@ -1,0 +1,87 @@
+"""ctypes view of the C ABI in include/attn_jvp.h (marshalling only)."""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libattn_jvp.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "attn_jvp.h")
+
+OK = 0
+ERR_INVALID_ARGUMENT = 1
+ERR_UNSUPPORTED = 2
+ERR_MISALIGNED = 3
+ERR_CUDA = 4
+ERR_DEVICE_TIMEOUT = 5
+ERR_NO_DEVICE = 6
+
+DTYPE_BF16 = 0
+DTYPE_F32 = 1
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int64), ("L", ctypes.c_int64), ("H", ctypes.c_int64),
+                ("d", ctypes.c_int64), ("dtype", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+
+class Mask(ctypes.Structure):
+    _fields_ = [("mode", ctypes.c_int32), ("chunk_tokens", ctypes.c_int32),
+                ("n_chunks", ctypes.c_int32)]
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def load() -> ctypes.CDLL:
+    """Load the in-tree CUDA library; raise if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"CUDA library not built: {LIB_PATH} is missing "
+                "(run `python -m attention_jvp_attn_b200.build`)")
+        lib = ctypes.CDLL(LIB_PATH)
+        vp = ctypes.c_void_p
+        lib.attn_jvp_fwd.argtypes = [ctypes.POINTER(Shape), vp, vp, vp, vp, vp, vp, Mask,
+                                     vp, vp, vp, vp]
+        lib.attn_jvp_fwd.restype = ctypes.c_int
+        lib.attn_jvp_fwd_host.argtypes = [ctypes.POINTER(Shape), vp, vp, vp, vp, vp, vp, Mask,
+                                          vp, vp, vp, vp, vp]
+        lib.attn_jvp_fwd_host.restype = ctypes.c_int
+        lib.attn_jvp_host_staging_bytes.argtypes = [ctypes.POINTER(Shape)]
+        lib.attn_jvp_host_staging_bytes.restype = ctypes.c_int64
+        lib.attn_jvp_sync_status.argtypes = [vp]
+        lib.attn_jvp_sync_status.restype = ctypes.c_int
+        lib.attn_jvp_status_string.argtypes = [ctypes.c_int]
+        lib.attn_jvp_status_string.restype = ctypes.c_char_p
+        lib.attn_jvp_unmasked_pairs.argtypes = [Mask]
+        lib.attn_jvp_unmasked_pairs.restype = ctypes.c_int64
+        lib.attn_jvp_schedule_tiles.argtypes = [Mask, ctypes.c_int64, ctypes.c_int32,
+                                                ctypes.c_int32, ctypes.c_int32,
+                                                ctypes.POINTER(ctypes.c_int32),
+                                                ctypes.POINTER(ctypes.c_uint8), ctypes.c_int32]
+        lib.attn_jvp_schedule_tiles.restype = ctypes.c_int32
+        lib.attn_jvp_version.argtypes = []
+        lib.attn_jvp_version.restype = ctypes.c_int32
+        _lib = lib
+        return lib
+
+
+def status_string(code: int) -> str:
+    return load().attn_jvp_status_string(code).decode()
+
+
+class AttnJvpError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: status {code} ({status_string(code)})")
+
+
+def check(code: int, where: str) -> None:
+    if code != OK:
+        raise AttnJvpError(code, where)

@@ -1,0 +1,343 @@
+// attn_jvp_api.cu - the C ABI declared in include/attn_jvp.h: argument
+// validation, TMA descriptor encoding, work ordering, launches, status words.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstddef>
+#include <cstring>
+#include <mutex>
+#include <numeric>
+#include <vector>
+
+#include "attn_jvp.h"
+#include "kernels.cuh"
+
+namespace {
+
+using ajvp::MaskSpec;
+
+constexpr int kMaxDevices = 64;
+constexpr int64_t kMaxSeq = int64_t(1) << 30;
+
+struct DeviceState {
+  bool ready = false;
+  int status_code = ATTN_JVP_OK;  // why the device is unusable, if it is
+  int sm_count = 0;
+  unsigned int* status = nullptr;  // device status word (bit 0: a bounded wait ran out)
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+// Per-device set-up, done once under the lock: checks the device is sm_100,
+// allocates the 4-byte status word and raises the kernels' shared-memory limit.
+int device_state(DeviceState** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
+    cudaGetLastError();
+    return ATTN_JVP_ERR_NO_DEVICE;
+  }
+  if (dev >= kMaxDevices) return ATTN_JVP_ERR_NO_DEVICE;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState& st = g_dev[dev];
+  if (!st.ready) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&st.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return ATTN_JVP_ERR_CUDA;
+    }
+    if (major != 10 || minor != 0) return ATTN_JVP_ERR_NO_DEVICE;  // built for sm_100a only
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+              cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !fn) {
+        cudaGetLastError();
+        return ATTN_JVP_ERR_CUDA;
+      }
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    if (cudaMalloc(&st.status, sizeof(unsigned int)) != cudaSuccess) {
+      cudaGetLastError();
+      st.status = nullptr;
+      return ATTN_JVP_ERR_CUDA;
+    }
+    if (cudaMemset(st.status, 0, sizeof(unsigned int)) != cudaSuccess ||
+        ajvp::tc_prepare(128) != cudaSuccess || ajvp::tc_prepare(64) != cudaSuccess ||
+        ajvp::simt_prepare(128) != cudaSuccess || ajvp::simt_prepare(64) != cudaSuccess) {
+      cudaGetLastError();
+      cudaFree(st.status);
+      st.status = nullptr;
+      return ATTN_JVP_ERR_CUDA;
+    }
+    st.ready = true;
+  }
+  *out = &st;
+  return ATTN_JVP_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int validate_mask(const attn_jvp_mask& m, int64_t* L_expected) {
+  if (m.mode != ATTN_JVP_MASK_TEACHER_FORCING && m.mode != ATTN_JVP_MASK_BLOCK_CAUSAL)
+    return ATTN_JVP_ERR_INVALID_ARGUMENT;
+  if (m.chunk_tokens < 1 || m.n_chunks < 1) return ATTN_JVP_ERR_INVALID_ARGUMENT;
+  const int64_t per = (m.mode == ATTN_JVP_MASK_TEACHER_FORCING) ? 2 : 1;
+  const int64_t L = per * int64_t(m.n_chunks) * int64_t(m.chunk_tokens);
+  if (L > kMaxSeq) return ATTN_JVP_ERR_INVALID_ARGUMENT;
+  *L_expected = L;
+  return ATTN_JVP_OK;
+}
+
+int validate(const attn_jvp_shape* s, attn_jvp_mask mask) {
+  if (!s) return ATTN_JVP_ERR_INVALID_ARGUMENT;
+  if (s->B < 1 || s->H < 1 || s->L < 1) return ATTN_JVP_ERR_INVALID_ARGUMENT;
+  if (s->dtype != ATTN_JVP_BF16 && s->dtype != ATTN_JVP_F32) return ATTN_JVP_ERR_UNSUPPORTED;
+  if (s->d != 64 && s->d != 128) return ATTN_JVP_ERR_UNSUPPORTED;
+  if (!(s->scale <= 0.f || std::isfinite(s->scale))) return ATTN_JVP_ERR_INVALID_ARGUMENT;
+  int64_t L = 0;
+  const int rc = validate_mask(mask, &L);
+  if (rc != ATTN_JVP_OK) return rc;
+  if (s->L != L) return ATTN_JVP_ERR_INVALID_ARGUMENT;
+  if (s->B > 65535 || s->H > 65535) return ATTN_JVP_ERR_INVALID_ARGUMENT;
+  // element counts must fit the kernels' 32-bit tile coordinates and 64-bit offsets
+  if (s->B * s->H * ((s->L + ajvp::kTcBlockM - 1) / ajvp::kTcBlockM) > int64_t(1) << 31)
+    return ATTN_JVP_ERR_INVALID_ARGUMENT;
+  return ATTN_JVP_OK;
+}
+
+float softmax_scale(const attn_jvp_shape* s) {
+  return s->scale > 0.f ? s->scale : 1.0f / std::sqrt(static_cast<float>(s->d));
+}
+
+bool encode_bf16_map(CUtensorMap* map, const void* base, const attn_jvp_shape* s, int box_rows) {
+  const cuuint64_t dims[4] = {cuuint64_t(s->d), cuuint64_t(s->H), cuuint64_t(s->L),
+                              cuuint64_t(s->B)};
+  const cuuint64_t strides[3] = {cuuint64_t(s->d) * 2, cuuint64_t(s->H * s->d) * 2,
+                                 cuuint64_t(s->L * s->H * s->d) * 2};
+  const cuuint32_t box[4] = {64, 1, cuuint32_t(box_rows), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+MaskSpec mask_spec(attn_jvp_mask m, int64_t L) {
+  MaskSpec ms;
+  ms.mode = m.mode;
+  ms.c = m.chunk_tokens;
+  ms.n = m.n_chunks;
+  ms.L = static_cast<int>(L);
+  return ms;
+}
+
+// Query tiles of one head, most key tiles first (stable among equals).
+int fill_order(const MaskSpec& ms, int n_qtiles, uint16_t* order) {
+  if (n_qtiles > ajvp::kMaxOrder) return 0;
+  std::vector<int> cost(n_qtiles), idx(n_qtiles);
+  for (int t = 0; t < n_qtiles; ++t) {
+    cost[t] = ajvp::make_tile_sched(ms, t, ajvp::kTcBlockM, ajvp::kTcBlockN).count();
+    idx[t] = t;
+  }
+  std::stable_sort(idx.begin(), idx.end(), [&](int a, int b) { return cost[a] > cost[b]; });
+  for (int r = 0; r < n_qtiles; ++r) order[r] = static_cast<uint16_t>(idx[r]);
+  return n_qtiles;
+}
+
+int launch_bf16(DeviceState* st, const attn_jvp_shape* s, const void* q, const void* k,
+                const void* v, const void* tq, const void* tk, const void* tv, attn_jvp_mask mask,
+                void* o, void* to, float* lse, cudaStream_t stream) {
+  static thread_local ajvp::TcParams p;  // large (order table): not on the stack
+  std::memset(&p, 0, offsetof(ajvp::TcParams, order));
+  if (!encode_bf16_map(&p.map_q, q, s, ajvp::kTcBlockM) ||
+      !encode_bf16_map(&p.map_k, k, s, ajvp::kTcBlockN) ||
+      !encode_bf16_map(&p.map_v, v, s, ajvp::kTcBlockN) ||
+      !encode_bf16_map(&p.map_tq, tq, s, ajvp::kTcBlockM) ||
+      !encode_bf16_map(&p.map_tk, tk, s, ajvp::kTcBlockN) ||
+      !encode_bf16_map(&p.map_tv, tv, s, ajvp::kTcBlockN))
+    return ATTN_JVP_ERR_CUDA;
+  p.o = o;
+  p.to = to;
+  p.lse = lse;
+  p.status = st->status;
+  p.B = static_cast<int>(s->B);
+  p.H = static_cast<int>(s->H);
+  p.L = static_cast<int>(s->L);
+  p.n_qtiles = static_cast<int>((s->L + ajvp::kTcBlockM - 1) / ajvp::kTcBlockM);
+  p.n_items = p.B * p.H * p.n_qtiles;
+  p.mask = mask_spec(mask, s->L);
+  const float sc = softmax_scale(s);
+  p.scale = sc;
+  p.scale_log2 = sc * 1.4426950408889634f;
+  p.order_len = fill_order(p.mask, p.n_qtiles, p.order);
+  const int grid = std::min(st->sm_count, p.n_items);
+  if (ajvp::tc_launch(static_cast<int>(s->d), p, grid, stream) != cudaSuccess)
+    return ATTN_JVP_ERR_CUDA;
+  return ATTN_JVP_OK;
+}
+
+int launch_f32(const attn_jvp_shape* s, const void* q, const void* k, const void* v,
+               const void* tq, const void* tk, const void* tv, attn_jvp_mask mask, void* o,
+               void* to, float* lse, cudaStream_t stream) {
+  ajvp::SimtParams p;
+  p.q = static_cast<const float*>(q);
+  p.k = static_cast<const float*>(k);
+  p.v = static_cast<const float*>(v);
+  p.tq = static_cast<const float*>(tq);
+  p.tk = static_cast<const float*>(tk);
+  p.tv = static_cast<const float*>(tv);
+  p.o = static_cast<float*>(o);
+  p.to = static_cast<float*>(to);
+  p.lse = lse;
+  p.B = static_cast<int>(s->B);
+  p.H = static_cast<int>(s->H);
+  p.L = static_cast<int>(s->L);
+  p.mask = mask_spec(mask, s->L);
+  const float sc = softmax_scale(s);
+  p.scale = sc;
+  p.scale_log2 = sc * 1.4426950408889634f;
+  if (ajvp::simt_launch(static_cast<int>(s->d), p, stream) != cudaSuccess) return ATTN_JVP_ERR_CUDA;
+  return ATTN_JVP_OK;
+}
+
+int64_t round256(int64_t x) { return (x + 255) & ~int64_t(255); }
+
+}  // namespace
+
+extern "C" {
+
+int attn_jvp_fwd(const attn_jvp_shape* shape, const void* q, const void* k, const void* v,
+                 const void* tq, const void* tk, const void* tv, attn_jvp_mask mask, void* o,
+                 void* to, float* lse, void* stream) {
+  int rc = validate(shape, mask);
+  if (rc != ATTN_JVP_OK) return rc;
+  const void* ptrs[9] = {q, k, v, tq, tk, tv, o, to, lse};
+  for (const void* ptr : ptrs)
+    if (!ptr) return ATTN_JVP_ERR_INVALID_ARGUMENT;
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return ATTN_JVP_ERR_MISALIGNED;
+  DeviceState* st = nullptr;
+  rc = device_state(&st);
+  if (rc != ATTN_JVP_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (shape->dtype == ATTN_JVP_BF16) return launch_bf16(st, shape, q, k, v, tq, tk, tv, mask, o, to, lse, s);
+  return launch_f32(shape, q, k, v, tq, tk, tv, mask, o, to, lse, s);
+}
+
+int64_t attn_jvp_host_staging_bytes(const attn_jvp_shape* shape) {
+  if (!shape || shape->B < 1 || shape->L < 1 || shape->H < 1 || shape->d < 1) return 0;
+  if (shape->dtype != ATTN_JVP_BF16 && shape->dtype != ATTN_JVP_F32) return 0;
+  const int64_t esz = shape->dtype == ATTN_JVP_BF16 ? 2 : 4;
+  const int64_t t = shape->B * shape->L * shape->H * shape->d * esz;
+  return 8 * round256(t) + round256(shape->B * shape->H * shape->L * 4);
+}
+
+int attn_jvp_fwd_host(const attn_jvp_shape* shape, const void* h_q, const void* h_k,
+                      const void* h_v, const void* h_tq, const void* h_tk, const void* h_tv,
+                      attn_jvp_mask mask, void* h_o, void* h_to, float* h_lse, void* d_buf,
+                      void* stream) {
+  int rc = validate(shape, mask);
+  if (rc != ATTN_JVP_OK) return rc;
+  const void* hp[9] = {h_q, h_k, h_v, h_tq, h_tk, h_tv, h_o, h_to, h_lse};
+  for (const void* ptr : hp)
+    if (!ptr) return ATTN_JVP_ERR_INVALID_ARGUMENT;
+  if (!d_buf) return ATTN_JVP_ERR_INVALID_ARGUMENT;
+  if (reinterpret_cast<uintptr_t>(d_buf) & 255u) return ATTN_JVP_ERR_MISALIGNED;
+  const int64_t esz = shape->dtype == ATTN_JVP_BF16 ? 2 : 4;
+  const int64_t tb = shape->B * shape->L * shape->H * shape->d * esz;
+  const int64_t lb = shape->B * shape->H * shape->L * 4;
+  char* base = static_cast<char*>(d_buf);
+  void* d[8];
+  for (int i = 0; i < 8; ++i) d[i] = base + i * round256(tb);
+  float* d_lse = reinterpret_cast<float*>(base + 8 * round256(tb));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const void* hin[6] = {h_q, h_k, h_v, h_tq, h_tk, h_tv};
+  for (int i = 0; i < 6; ++i)
+    if (cudaMemcpyAsync(d[i], hin[i], tb, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+      cudaGetLastError();
+      return ATTN_JVP_ERR_CUDA;
+    }
+  rc = attn_jvp_fwd(shape, d[0], d[1], d[2], d[3], d[4], d[5], mask, d[6], d[7], d_lse, stream);
+  if (rc != ATTN_JVP_OK) return rc;
+  if (cudaMemcpyAsync(h_o, d[6], tb, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaMemcpyAsync(h_to, d[7], tb, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaMemcpyAsync(h_lse, d_lse, lb, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_JVP_ERR_CUDA;
+  }
+  return attn_jvp_sync_status(stream);
+}
+
+int attn_jvp_sync_status(void* stream) {
+  DeviceState* st = nullptr;
+  int rc = device_state(&st);
+  if (rc != ATTN_JVP_OK) return rc;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_JVP_ERR_CUDA;
+  }
+  unsigned int word = 0;
+  if (cudaMemcpy(&word, st->status, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_JVP_ERR_CUDA;
+  }
+  if (word != 0) {
+    cudaMemset(st->status, 0, sizeof(unsigned int));
+    return ATTN_JVP_ERR_DEVICE_TIMEOUT;
+  }
+  return ATTN_JVP_OK;
+}
+
+const char* attn_jvp_status_string(int status) {
+  switch (status) {
+    case ATTN_JVP_OK: return "ok";
+    case ATTN_JVP_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case ATTN_JVP_ERR_UNSUPPORTED: return "unsupported dtype or head dim";
+    case ATTN_JVP_ERR_MISALIGNED: return "pointer not aligned";
+    case ATTN_JVP_ERR_CUDA: return "CUDA error";
+    case ATTN_JVP_ERR_DEVICE_TIMEOUT: return "device wait timed out; outputs invalid";
+    case ATTN_JVP_ERR_NO_DEVICE: return "no usable sm_100 device";
+    default: return "unknown status";
+  }
+}
+
+int64_t attn_jvp_unmasked_pairs(attn_jvp_mask mask) {
+  int64_t L = 0;
+  if (validate_mask(mask, &L) != ATTN_JVP_OK) return -1;
+  const int64_t c = mask.chunk_tokens, n = mask.n_chunks;
+  const int64_t tf = c * c * n * (n + 1);
+  return mask.mode == ATTN_JVP_MASK_TEACHER_FORCING ? tf : tf / 2;
+}
+
+int32_t attn_jvp_schedule_tiles(attn_jvp_mask mask, int64_t L, int32_t block_m, int32_t block_n,
+                                int32_t q_tile, int32_t* tiles, uint8_t* full, int32_t cap) {
+  int64_t Lx = 0;
+  if (validate_mask(mask, &Lx) != ATTN_JVP_OK || Lx != L) return -1;
+  if (block_m < 1 || block_n < 1 || q_tile < 0 || cap < 0) return -1;
+  if (int64_t(q_tile) * block_m >= L) return -1;
+  if ((tiles == nullptr || full == nullptr) && cap > 0) return -1;
+  const MaskSpec ms = mask_spec(mask, L);
+  const ajvp::TileSched s = ajvp::make_tile_sched(ms, q_tile, block_m, block_n);
+  const int n = s.count();
+  for (int i = 0; i < n && i < cap; ++i) {
+    tiles[i] = s.tile(i);
+    full[i] = s.full(s.tile(i)) ? 1 : 0;
+  }
+  return n;
+}
+
+int32_t attn_jvp_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,55 @@
+// kernels.cuh - launch parameters shared by the C ABI and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "mask_schedule.cuh"
+
+namespace ajvp {
+
+// ---- bf16 tensor-core kernel (tcgen05 / TMEM / TMA) ----
+constexpr int kTcBlockM = 128;   // query rows per tile (one TMEM lane per row)
+constexpr int kTcBlockN = 128;   // keys per tile
+constexpr int kTcThreads = 192;  // warps 0-3 softmax+epilogue, 4 TMA producer, 5 MMA issuer
+constexpr int kMaxOrder = 4096;  // longest-first query-tile order table capacity
+
+struct TcParams {
+  CUtensorMap map_q, map_k, map_v, map_tq, map_tk, map_tv;  // [B, L, H, d] bf16, 128B swizzle
+  void* o;
+  void* to;
+  float* lse;
+  unsigned int* status;
+  int B, H, L;
+  int n_qtiles;  // ceil(L / 128)
+  int n_items;   // B * H * n_qtiles
+  MaskSpec mask;
+  float scale_log2;  // s * log2(e)
+  float scale;       // s
+  int order_len;     // n_qtiles if `order` is filled, else 0 (reverse index order)
+  uint16_t order[kMaxOrder];
+};
+
+size_t tc_smem_bytes(int d);
+cudaError_t tc_prepare(int d);  // sets the dynamic shared-memory limit (once per device)
+cudaError_t tc_launch(int d, const TcParams& p, int grid, cudaStream_t stream);
+
+// ---- fp32 CUDA-core kernel ----
+constexpr int kSimtBlockQ = 32;
+constexpr int kSimtBlockK = 32;
+constexpr int kSimtThreads = 256;
+
+struct SimtParams {
+  const float *q, *k, *v, *tq, *tk, *tv;
+  float *o, *to, *lse;
+  int B, H, L;
+  MaskSpec mask;
+  float scale_log2, scale;
+};
+
+size_t simt_smem_bytes(int d);
+cudaError_t simt_prepare(int d);
+cudaError_t simt_launch(int d, const SimtParams& p, cudaStream_t stream);
+
+}  // namespace ajvp

@@ -126,18 +126,18 @@ def make_inputs(w: Workload, device="cpu", seed: Optional[int] = None,
 def sample_rows(w: Workload, n_random: int = 256, seed: int = 7,
                 tile: int = 128) -> List[int]:
     """Query rows worth checking one by one on a large workload: first and
-    last row of every chunk (clean and noisy), both sides of every `tile`
-    boundary, the ragged tail, and `n_random` seeded random rows."""
+    last row of every chunk (clean and noisy), the rows on both sides of the
+    `tile` boundaries around every chunk boundary (where tiles are partial),
+    the ragged tail, and `n_random` seeded random rows."""
     L, c = w.L, w.chunk_tokens
     rows = set()
-    n_blocks = L // c
-    for j in range(n_blocks):
-        rows.add(j * c)
-        rows.add(j * c + c - 1)
-    for t in range(tile, L, tile):
-        rows.add(t - 1)
-        rows.add(t)
-    rows.add(L - 1)
+    for j in range(L // c):
+        p = j * c
+        rows.update((p, p + c - 1))
+        t = p // tile
+        for q in (t * tile - 1, t * tile, (t + 1) * tile - 1, (t + 1) * tile):
+            rows.add(q)
+    rows.update((L - 1, (L - 1) // tile * tile, (L - 1) // tile * tile - 1))
     g = torch.Generator().manual_seed(seed)
     rows.update(torch.randint(0, L, (n_random,), generator=g).tolist())
     return sorted(r for r in rows if 0 <= r < L)

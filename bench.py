@@ -1,0 +1,396 @@
+"""Benchmark: custom-mask attention forward + JVP on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step is one call of the fused attention+JVP kernel over one batch of the
+workload (default: frame-wise teacher forcing, B=1, H=12, d=128, 21 chunks x
+1560 tokens packed clean|noisy, L=65520, bf16), inputs resident in HBM. The
+metric is effective TFLOP/s over admissible (unmasked) query-key pairs,
+12 d FLOPs per pair. Each rank runs its own replica of the workload (weak
+scaling, no collective on the data path); rank 0 prints one JSON line.
+
+--impl reference times the float64 CPU oracle on the host cores instead (a
+bounded sample of the same workload per step) and prints the same line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import glob
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+
+
+def _env_int(name, default):
+    try:
+        return int(os.environ.get(name, default))
+    except ValueError:
+        return default
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "attention_jvp_attn_b200", "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(os.path.basename(p).encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(workload)
+    if not e or e.get("kernel_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            self.proc.wait()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        smax = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for name, val in zip(names, r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(name)
+        power = [num(r[3]) for r in rows if num(r[3]) is not None]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(rows),
+                "power_w_max": max(power) if power else None}
+
+
+def workload_by_name(name):
+    from attention_jvp_attn_b200 import inputs as wl
+    if name not in wl.WORKLOADS:
+        raise SystemExit(f"unknown workload {name}; choose from {sorted(wl.WORKLOADS)}")
+    return wl.WORKLOADS[name]
+
+
+def flops_per_step(w) -> int:
+    from attention_jvp_attn_b200 import inputs as wl
+    c, n = w.chunk_tokens, w.n_chunks
+    pairs = c * c * n * (n + 1) // (1 if w.mode == wl.TEACHER_FORCING else 2)
+    return 12 * w.d * pairs * w.B * w.H
+
+
+def workload_config(w, n_gpus):
+    from attention_jvp_attn_b200 import inputs as wl
+    return {"workload": w.name, "mask": wl.MODE_NAMES[w.mode], "B": w.B, "H": w.H, "d": w.d,
+            "n_chunks": w.n_chunks, "chunk_tokens": w.chunk_tokens, "seq_len": w.L,
+            "global_batch": w.B * n_gpus, "parallelism": f"{n_gpus} independent replicas",
+            "l2": f"no flush: inputs {w.input_bytes() / 1e9:.2f} GB > 126 MB L2"}
+
+
+# --------------------------------------------------------------------------- oracle timing
+
+def oracle_sample(w, budget_s: float, seed: int = 0):
+    """Time the float64 oracle on seeded random query rows of head 0 of the
+    workload (CPU inputs drawn from the same generator recipe), growing the
+    sample until about `budget_s` seconds of work. Returns (effective FLOP/s,
+    rows, seconds, threads)."""
+    import numpy as np
+    import torch
+    from attention_jvp_attn_b200 import inputs as wl
+    from oracle import attn_jvp_oracle as orc
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        threads = max((i.get("num_threads", 1) for i in info), default=1)
+    except Exception:
+        threads = 1
+    g = torch.Generator().manual_seed(w.seed)
+    one = (w.L, w.d)
+    x = [(torch.randn(one, generator=g) * s).to(torch.bfloat16 if w.dtype == "bf16" else torch.float32)
+         for s in w.stds]
+    x64 = [orc._as64(t) for t in x]
+    rng = np.random.default_rng(seed)
+    total_pairs, total_t, rows_done = 0, 0.0, 0
+    batch = 16
+    while total_t < budget_s:
+        rows = rng.integers(0, w.L, size=batch)
+        t0 = time.perf_counter()
+        orc.attn_jvp_rows(*x64, w.mode, w.chunk_tokens, w.n_chunks, w.scale, rows)
+        total_t += time.perf_counter() - t0
+        M = orc.allowed(w.mode, w.chunk_tokens, w.n_chunks, rows[:, None], np.arange(w.L)[None, :])
+        total_pairs += int(M.sum())
+        rows_done += batch
+        if total_t < budget_s / 4:
+            batch *= 2
+    return 12 * w.d * total_pairs / total_t, rows_done, total_t, threads
+
+
+def run_reference(args):
+    rank = _env_int("RANK", 0)
+    world = _env_int("WORLD_SIZE", 1)
+    if rank != 0:
+        return 0
+    w = workload_by_name(args.workload)
+    for _ in range(args.warmup):
+        oracle_sample(w, budget_s=0.5)
+    vals, secs, rows_all = [], 0.0, 0
+    threads = 1
+    for _ in range(args.steps):
+        v, rows, t, threads = oracle_sample(w, budget_s=args.ref_budget)
+        vals.append(v)
+        secs += t
+        rows_all += rows
+    value = statistics.mean(vals) / 1e12
+    sample = (f"{rows_all} seeded random query rows of head 0 over {args.steps} steps "
+              f"(about {args.ref_budget:.0f} s each), float64 dense rows masked by the explicit "
+              f"predicate; effective FLOPs = 12 d x admissible pairs of the sampled rows")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * flops_per_step(w) / (value * 1e12),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(w, 1),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+METRIC = "attention+JVP effective TFLOP/s (unmasked pairs) and % of B200 bf16 peak"
+
+
+# --------------------------------------------------------------------------- GPU arm
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+    import attention_jvp_attn_b200 as aj
+    from attention_jvp_attn_b200 import inputs as wl
+
+    rank = _env_int("RANK", 0)
+    world = _env_int("WORLD_SIZE", 1)
+    local = _env_int("LOCAL_RANK", 0)
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    w = workload_by_name(args.workload)
+    x = wl.make_inputs(w, device=dev, seed=w.seed + 7919 * rank)
+    B, L, H, d = w.B, w.L, w.H, w.d
+    dt = x["q"].dtype
+    o = torch.empty_like(x["q"])
+    to = torch.empty_like(x["q"])
+    lse = torch.empty((B, H, L), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        aj.attn_jvp(x["q"], x["k"], x["v"], x["tq"], x["tk"], x["tv"], w.mode, w.chunk_tokens,
+                    w.n_chunks, w.scale, out=(o, to, lse))
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    st = aj.sync_status(dev)
+    if st != 0:
+        raise SystemExit(f"device status {st} after warm-up")
+
+    clocks = ClockSampler(local)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.25)  # let the sampler start before the timed region
+    t_begin = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_begin.record(stream)
+    for i in range(args.steps):
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop()
+    st = aj.sync_status(dev)
+    if st != 0:
+        raise SystemExit(f"device status {st} after timed steps")
+    total_ms = t_begin.elapsed_time(t_end)
+    launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    if world > 1:
+        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms_per_step = total_ms / args.steps
+    flops = flops_per_step(w)
+    value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
+
+    # end to end through the host-buffer C-ABI entry point (pinned host memory)
+    e2e = None
+    if not args.no_e2e:
+        xh = {k: v.cpu().pin_memory() for k, v in x.items()}
+        oh = torch.empty((B, L, H, d), dtype=dt).pin_memory()
+        toh = torch.empty((B, L, H, d), dtype=dt).pin_memory()
+        lseh = torch.empty((B, H, L), dtype=torch.float32).pin_memory()
+        staging = torch.empty(aj.host_staging_bytes(B, L, H, d, dt), dtype=torch.uint8, device=dev)
+
+        def e2e_step():
+            aj.attn_jvp_host(xh["q"], xh["k"], xh["v"], xh["tq"], xh["tk"], xh["tv"], w.mode,
+                             w.chunk_tokens, w.n_chunks, staging, (oh, toh, lseh), w.scale, dev)
+        e2e_step()
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e2e_ms = float(tt.item())
+        tensor_bytes = B * L * H * d * x["q"].element_size()
+        e2e = {"value": world * flops * args.e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": e2e_ms / args.e2e_steps,
+               "h2d_bytes_per_step": 6 * tensor_bytes,
+               "d2h_bytes_per_step": 2 * tensor_bytes + B * H * L * 4}
+        del xh, oh, toh, lseh, staging
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    avg_launch_ms = sum(launch_ms) / len(launch_ms)
+    achieved = flops / (avg_launch_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": load_traffic(w.name),
+                "peak_source": f"{peak_src} bf16 dense burst",
+                "sustained_peak": float(peaks.get("bf16_tflops_sustained",
+                                                  FALLBACK_PEAKS["bf16_tflops_sustained"])),
+                "kernel": "attn_jvp_tc_kernel<128>" if d == 128 else "attn_jvp_tc_kernel<64>",
+                "flops_per_launch": flops, "avg_launch_ms": avg_launch_ms}
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        v, rows, secs, threads = oracle_sample(w, budget_s=args.cpu_budget)
+        cpu = {"value": v / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": (f"{rows} seeded random query rows of one head, {secs:.1f} s of float64 "
+                          f"oracle work; effective FLOPs = 12 d x admissible pairs of those rows")}
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "pct_of_peak": 100.0 * value / world / peak,
+            "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": workload_config(w, world), "roofline": roofline, "cpu_baseline": cpu,
+            "e2e": e2e, "gpu_launches": args.steps, "clocks": clk}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="framewise_tf_bf16")
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--ref-budget", type=float, default=6.0)
+    args = ap.parse_args()
+    if args.warmup < 0 or args.steps < 1:
+        raise SystemExit("need --steps >= 1 and --warmup >= 0")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

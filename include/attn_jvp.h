@@ -1,0 +1,192 @@
+/*
+ * attn_jvp.h - C ABI of the B200 (sm_100a) custom-mask attention + JVP library.
+ *
+ * The operation (Causal-rCM summary page, App. B "FlashAttention-2 JVP Kernel
+ * with Custom Masks"): for queries Q, keys K, values V and tangents tQ, tK,
+ * tV, with softmax scale s and an additive mask M (0 where a query may attend
+ * to a key, -inf elsewhere),
+ *
+ *     S  = s Q K^T + M,        P  = softmax(S) (row-wise),    O = P V
+ *     tS = s (tQ K^T + Q tK^T)
+ *     tP = P * (tS - rowsum(P * tS))                (elementwise *)
+ *     tO = tP V + P tV
+ *     LSE_i = log sum_j exp(S_ij)                   (natural log)
+ *
+ * Masked entries receive no tangent, because the discrete mask has none
+ * (App. B); the tangent uses exactly the primal masked operator and the same
+ * sparse schedule (App. B). The library returns the primal output, the
+ * log-sum-exp values and the tangent output (App. B, last item).
+ *
+ * Masks are given as {mode, chunk_tokens c, n_chunks n}:
+ *   ATTN_JVP_MASK_TEACHER_FORCING: the packed sequence [clean chunks | noisy
+ *     chunks], L = 2 n c (Causal-rCM page, section 3 "Continuous-time
+ *     consistency", TF-masked packed forward; Causal Forcing summary page,
+ *     section 2, clean and noisy videos concatenated under a causal mask).
+ *     A clean query in chunk j attends to clean chunks <= j. A noisy query in
+ *     chunk i attends to clean chunks < i and to its own noisy chunk.
+ *   ATTN_JVP_MASK_BLOCK_CAUSAL: L = n c; a query in chunk j attends to
+ *     chunks <= j (Causal-rCM page, section 2 "Autoregressive video
+ *     diffusion": causal across temporal blocks, full attention inside one).
+ * Attention inside one chunk is full in both modes.
+ *
+ * Layout: q, k, v, tq, tk, tv, o, to are dense row-major [B, L, H, d] arrays
+ * (d innermost) of the element type `dtype`; lse is a dense [B, H, L] float
+ * array. All of them are DEVICE pointers of the current CUDA device unless a
+ * function says otherwise.
+ *
+ * Ownership: the caller owns every buffer; the library never frees or keeps
+ * a caller pointer after the call returns (work is stream-ordered: buffers
+ * must stay valid until the stream reaches the launched work). The library
+ * keeps, per device, a small status word and cached tensor-map descriptors;
+ * it allocates nothing else. Outputs must not overlap inputs or each other.
+ *
+ * Errors: every function returns an int status (ATTN_JVP_OK = 0 on success)
+ * and never throws. Argument errors are detected on the host before anything
+ * is launched. attn_jvp_fwd does not synchronize; device-side faults of the
+ * launched work (a bounded wait that ran out) are reported later by
+ * attn_jvp_sync_status.
+ *
+ * Threading: functions may be called from several host threads; the cached
+ * descriptors are protected by a lock.
+ */
+#ifndef ATTN_JVP_H_
+#define ATTN_JVP_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ---------------------------------------------------- */
+enum {
+  ATTN_JVP_OK = 0,
+  ATTN_JVP_ERR_INVALID_ARGUMENT = 1, /* null pointer, bad size, L inconsistent with the mask */
+  ATTN_JVP_ERR_UNSUPPORTED = 2,      /* dtype or head_dim the kernels do not implement */
+  ATTN_JVP_ERR_MISALIGNED = 3,       /* a pointer is not 16-byte aligned */
+  ATTN_JVP_ERR_CUDA = 4,             /* a CUDA runtime or driver call failed */
+  ATTN_JVP_ERR_DEVICE_TIMEOUT = 5,   /* a kernel's bounded wait ran out; the outputs are invalid */
+  ATTN_JVP_ERR_NO_DEVICE = 6         /* no usable sm_100 device */
+};
+
+/* ---- mask ------------------------------------------------------------ */
+typedef enum {
+  ATTN_JVP_MASK_TEACHER_FORCING = 0,
+  ATTN_JVP_MASK_BLOCK_CAUSAL = 1
+} attn_jvp_mask_mode;
+
+typedef struct {
+  int32_t mode;         /* attn_jvp_mask_mode */
+  int32_t chunk_tokens; /* c >= 1: tokens per chunk (one latent frame = 1560 in Wan2.1) */
+  int32_t n_chunks;     /* n >= 1 */
+} attn_jvp_mask;
+
+/* ---- problem --------------------------------------------------------- */
+typedef enum {
+  ATTN_JVP_BF16 = 0, /* bf16 inputs/outputs, fp32 accumulation, tensor cores */
+  ATTN_JVP_F32 = 1   /* fp32 inputs/outputs, fp32 arithmetic on CUDA cores */
+} attn_jvp_dtype;
+
+typedef struct {
+  int64_t B;     /* batch >= 1 */
+  int64_t L;     /* sequence length: 2 n c (teacher forcing) or n c (block causal) */
+  int64_t H;     /* heads >= 1 */
+  int64_t d;     /* head dim: 64 or 128 */
+  int32_t dtype; /* attn_jvp_dtype */
+  float scale;   /* softmax scale s; <= 0 selects 1/sqrt(d) */
+} attn_jvp_shape;
+
+/*
+ * attn_jvp_fwd - O, tO and LSE of masked softmax attention and its JVP in one
+ * fused pass (App. B: same online-softmax pass and shared rescaling for the
+ * primal and tangent accumulators; fully masked key tiles are skipped).
+ *
+ *   shape   problem sizes and element type (host pointer, read during the call)
+ *   q..tv   device inputs, [B, L, H, d] of `shape->dtype`, 16-byte aligned
+ *   mask    mask mode and chunking; L must equal 2 n c or n c
+ *   o, to   device outputs, [B, L, H, d] of `shape->dtype`, 16-byte aligned
+ *   lse     device output, [B, H, L] float (natural-log log-sum-exp of the
+ *           scaled, masked scores)
+ *   stream  cudaStream_t to launch on (NULL = legacy default stream)
+ *
+ * Returns ATTN_JVP_OK after enqueueing the work, or an error code with
+ * nothing launched. The call does not synchronize with the device.
+ */
+int attn_jvp_fwd(const attn_jvp_shape* shape,
+                 const void* q, const void* k, const void* v,
+                 const void* tq, const void* tk, const void* tv,
+                 attn_jvp_mask mask,
+                 void* o, void* to, float* lse,
+                 void* stream);
+
+/*
+ * attn_jvp_fwd_host - the same operation on HOST buffers: copies the six
+ * inputs host->device, runs attn_jvp_fwd, copies O, tO and LSE device->host
+ * and waits for the stream. Host buffers should be pinned (page-locked) for
+ * the copies to run at full speed; pageable memory also works.
+ *
+ *   h_q..h_tv  host inputs, [B, L, H, d]
+ *   h_o, h_to  host outputs, [B, L, H, d];  h_lse host output [B, H, L]
+ *   d_buf      caller-owned device staging buffer of at least
+ *              attn_jvp_host_staging_bytes(shape) bytes, 256-byte aligned
+ *   stream     stream for the copies and the kernel
+ *
+ * Returns the status of the whole sequence, including any device fault
+ * (the call synchronizes on `stream`).
+ */
+int attn_jvp_fwd_host(const attn_jvp_shape* shape,
+                      const void* h_q, const void* h_k, const void* h_v,
+                      const void* h_tq, const void* h_tk, const void* h_tv,
+                      attn_jvp_mask mask,
+                      void* h_o, void* h_to, float* h_lse,
+                      void* d_buf, void* stream);
+
+/* Bytes of device staging attn_jvp_fwd_host needs for `shape` (0 on a bad shape). */
+int64_t attn_jvp_host_staging_bytes(const attn_jvp_shape* shape);
+
+/*
+ * attn_jvp_sync_status - synchronizes `stream`, then reports and clears the
+ * device status word of the current device: ATTN_JVP_ERR_DEVICE_TIMEOUT if a
+ * kernel gave up on a bounded wait since the last call, ATTN_JVP_ERR_CUDA if
+ * the stream reported an error, else ATTN_JVP_OK.
+ */
+int attn_jvp_sync_status(void* stream);
+
+/* Static, NUL-terminated description of a status code. */
+const char* attn_jvp_status_string(int status);
+
+/* ---- host-side helpers (need no GPU) ---------------------------------- */
+
+/* Number of admissible (query, key) pairs per (batch, head):
+ * c^2 n (n+1) for teacher forcing, c^2 n (n+1) / 2 for block causal; -1 on a
+ * bad mask. Effective FLOPs of one call are 12 d B H times this. */
+int64_t attn_jvp_unmasked_pairs(attn_jvp_mask mask);
+
+/*
+ * attn_jvp_schedule_tiles - the key-tile schedule the bf16 kernel runs for one
+ * query tile (App. B: masks as query groups with admissible key ranges; the
+ * same sparse schedule drives primal and tangent scores).
+ *
+ *   mask, L       mask and sequence length (validated as for attn_jvp_fwd)
+ *   block_m/_n    query / key tile sizes (rows / columns)
+ *   q_tile        query tile index, 0 <= q_tile < ceil(L / block_m)
+ *   tiles, full   caller arrays of `cap` entries: key tile indices in visit
+ *                 order, and 1 where every (query, key) pair of the tile is
+ *                 admissible (no element mask needed), 0 where it is partial
+ *   cap           capacity of both arrays
+ *
+ * Returns the number of key tiles (>= 0; entries beyond `cap` are not
+ * written) or -1 on a bad argument. Key tiles not listed are fully masked.
+ */
+int32_t attn_jvp_schedule_tiles(attn_jvp_mask mask, int64_t L, int32_t block_m,
+                                int32_t block_n, int32_t q_tile,
+                                int32_t* tiles, uint8_t* full, int32_t cap);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int32_t attn_jvp_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_JVP_H_ */

@@ -22,10 +22,11 @@
 // m_new)) when a tile's max exceeds it by more than kRescaleTau: every p stays
 // <= 2^kRescaleTau and the final normalisation by l is exact.
 //
-// Warp roles (192 threads, one CTA per SM, persistent over work items):
-//   warps 0-3  softmax + epilogue, thread i owns query row / TMEM lane i
-//   warp  4    TMA producer (one thread): Q,tQ per item; K,tK,V,tV per key tile
-//   warp  5    MMA issuer (one thread), TMEM allocator
+// Warp roles (320 threads, one CTA per SM, persistent over work items):
+//   warps 0-7  softmax + epilogue: two warpgroups, each owning half of the
+//              key columns of a tile (and half of the output columns)
+//   warp  8    TMA producer (one thread): Q,tQ per item; K,tK,tV,V per key tile
+//   warp  9    MMA issuer (one thread), TMEM allocator
 // Work items (batch, head, query tile) are ordered head-major so that CTAs
 // running at the same time share one head's keys in L2, and, within a head,
 // longest first; CTA c takes items c, 2G-1-c, 2G+c, ... of that list.
@@ -49,8 +50,11 @@ struct TcCfg {
   static constexpr int QBYTES = BM * D * 2;       // bytes of the Q (or tQ) tile
   static constexpr int NSLOT = (D == 128) ? 5 : 10;
   static constexpr int DATA = 2 * QBYTES + NSLOT * TILE;
-  static constexpr int NBAR = 2 * NSLOT + 8;
-  static constexpr int BYTES = 1024 + DATA + NBAR * 8 + 16;
+  static constexpr int XCH = 2 * BM * 4;          // row-statistics exchange, [2][BM] floats
+  static constexpr int NBAR = 2 * NSLOT + 9 + 8;
+  static constexpr int BYTES = 1024 + DATA + XCH + NBAR * 8 + 16;
+  static constexpr int HALF = BN / 2;             // key columns per softmax warpgroup
+  static constexpr int DH = D / 2;                // output columns per softmax warpgroup
   static constexpr uint32_t TM_S = 0;
   static constexpr uint32_t TM_TS = 128;
   static constexpr uint32_t TM_A = 256;
@@ -76,12 +80,29 @@ __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t base, int ks) {
   return smem_desc_sw128(base + ks * 16 * 128, BN * 128, 1024);
 }
 
+// bf16 P (or U) in TMEM: warpgroup h packs keys [64 h, 64 h + 64) into the
+// first 32 of its own 64 score columns, so key k sits at column
+// 64 (k / 64) + (k % 64) / 2. K-step ks of the value MMAs covers keys
+// [16 ks, 16 ks + 16).
+__device__ __forceinline__ uint32_t tmem_a_operand(uint32_t base, int ks) {
+  return base + 64 * (ks >> 2) + (ks & 3) * 8;
+}
+
 struct WorkItem {
   int b, h, qt;
 };
 
 __device__ __forceinline__ int item_position(int k, int cta, int G) {
   return (k & 1) ? k * G + (G - 1 - cta) : k * G + cta;
+}
+
+// First work item of this CTA at round >= k (k is advanced to it).
+__device__ __forceinline__ bool next_item(const TcParams& p, int cta, int G, int& k, int& pos) {
+  for (; k * G < p.n_items; ++k) {
+    pos = item_position(k, cta, G);
+    if (pos < p.n_items) return true;
+  }
+  return false;
 }
 
 __device__ __forceinline__ WorkItem decode_item(const TcParams& p, int pos) {
@@ -103,7 +124,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
   uint8_t* sQ = smem;
   uint8_t* sTQ = smem + C::QBYTES;
   uint8_t* sRing = smem + 2 * C::QBYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::DATA);
+  float* xch = reinterpret_cast<float*>(smem + C::DATA);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::DATA + C::XCH);
   uint64_t* full = bars;
   uint64_t* empty = bars + C::NSLOT;
   uint64_t* q_full = bars + 2 * C::NSLOT + 0;
@@ -113,7 +135,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
   uint64_t* p_full = bars + 2 * C::NSLOT + 4;
   uint64_t* u_full = bars + 2 * C::NSLOT + 5;
   uint64_t* acc_full = bars + 2 * C::NSLOT + 6;
-  uint64_t* drain = bars + 2 * C::NSLOT + 7;
+  uint64_t* uv_done = bars + 2 * C::NSLOT + 7;
+  uint64_t* drain = bars + 2 * C::NSLOT + 8;
+  uint64_t* xa = bars + 2 * C::NSLOT + 9;   // [4] row-statistics exchange, first half
+  uint64_t* xb = bars + 2 * C::NSLOT + 13;  // [4] second half
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -131,14 +156,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
     mbar_init(q_empty, 1);
     mbar_init(s_full, 1);
     mbar_init(ts_full, 1);
-    mbar_init(p_full, 4);
-    mbar_init(u_full, 4);
+    mbar_init(p_full, 8);
+    mbar_init(u_full, 8);
     mbar_init(acc_full, 1);
+    mbar_init(uv_done, 1);
     mbar_init(drain, 1);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&xa[i], 64);
+      mbar_init(&xb[i], 64);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, C::TM_COLS);
     tmem_relinquish();
   }
@@ -147,8 +177,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
+    // Load order per key tile matches the MMA issuer's first use: K, tK, tV, V.
     if (lane == 0) {
       tma_prefetch_desc(&p.map_q);
       tma_prefetch_desc(&p.map_k);
@@ -157,12 +188,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
       tma_prefetch_desc(&p.map_tk);
       tma_prefetch_desc(&p.map_tv);
       const uint64_t keep = l2_policy_evict_last();
-      const CUtensorMap* kv_maps[4] = {&p.map_k, &p.map_tk, &p.map_v, &p.map_tv};
+      const CUtensorMap* kv_maps[4] = {&p.map_k, &p.map_tk, &p.map_tv, &p.map_v};
       uint32_t ctr = 0, q_issued = 0, q_ph = 0;
       bool ok = true;
-      for (int k = 0; ok && k * G < p.n_items; ++k) {
-        const int pos = item_position(k, cta, G);
-        if (pos >= p.n_items) continue;
+      int k = 0, pos = 0;
+      while (ok && next_item(p, cta, G, k, pos)) {
+        ++k;
         const WorkItem w = decode_item(p, pos);
         if (q_issued > 0) {
           if (!mbar_wait(q_empty, q_ph, abort_flag, p.status)) { ok = false; break; }
@@ -204,77 +235,145 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
       }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
+    // Per key tile g (slots 4g..4g+3 hold K_g, tK_g, tV_g, V_g), in issue order:
+    //   T (+)= P_g tV_g,  A (+)= P_g V_g,  S_{g+1} = Q K_{g+1}^T,
+    //   T += U_g V_g,  tS'_{g+1} = tQ K_{g+1}^T + Q tK_{g+1}^T
+    // so the softmax warps compute U_g while P_g's products and S_{g+1} run,
+    // and P_{g+1} while U_g V_g and tS'_{g+1} run. tcgen05.mma from one thread
+    // execute in order, so S_{g+1} (over P_g's columns) follows every read of
+    // P_g and tS'_{g+1} (over U_g's columns) follows U_g V_g.
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(C::BM, C::BN, 0);
       const uint32_t idesc_v = idesc_bf16_f32(C::BM, D, 1);
       const uint32_t aQ = smem_u32(sQ), aTQ = smem_u32(sTQ), aRing = smem_u32(sRing);
-      uint32_t ctr = 0, q_ph = 0, p_ph = 0, u_ph = 0;
+      auto slot_addr = [&](uint32_t c) { return aRing + (c % C::NSLOT) * C::TILE; };
+      auto slot_ph = [&](uint32_t c) { return (c / C::NSLOT) & 1; };
+      uint32_t q_ph = 0, p_ph = 0, u_ph = 0;
       bool ok = true;
-      for (int k = 0; ok && k * G < p.n_items; ++k) {
-        const int pos = item_position(k, cta, G);
-        if (pos >= p.n_items) continue;
-        const WorkItem w = decode_item(p, pos);
-        if (!mbar_wait(q_full, q_ph, abort_flag, p.status)) { ok = false; break; }
+      int k = 0, pos = 0;
+      if (next_item(p, cta, G, k, pos)) {
+        ++k;
+        WorkItem w = decode_item(p, pos);
+        TileSched sch = make_tile_sched(p.mask, w.qt, C::BM, C::BN);
+        int cnt = sch.count(), idx = 0;
+        uint32_t g = 0;
+        // prologue: scores of the first tile
+        ok = mbar_wait(q_full, q_ph, abort_flag, p.status);
         q_ph ^= 1;
-        tc_fence_after();
-        const TileSched sch = make_tile_sched(p.mask, w.qt, C::BM, C::BN);
-        const int cnt = sch.count();
-        for (int idx = 0; idx < cnt; ++idx, ctr += 4) {
-          const uint32_t sK = ctr % C::NSLOT, sTK = (ctr + 1) % C::NSLOT;
-          const uint32_t sV = (ctr + 2) % C::NSLOT, sTV = (ctr + 3) % C::NSLOT;
-          const uint32_t aK = aRing + sK * C::TILE, aTK = aRing + sTK * C::TILE;
-          const uint32_t aV = aRing + sV * C::TILE, aTV = aRing + sTV * C::TILE;
-          // S = Q K^T
-          if (!mbar_wait(&full[sK], (ctr / C::NSLOT) & 1, abort_flag, p.status)) { ok = false; break; }
+        if (ok) ok = mbar_wait(&full[0], 0, abort_flag, p.status);
+        if (ok) {
           tc_fence_after();
+          const uint32_t aK = slot_addr(0);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
             umma_ss(tmem + C::TM_S, desc_kmajor(aQ, C::BM, kk), desc_kmajor(aK, C::BN, kk), idesc_s,
                     kk > 0);
           umma_commit(s_full);
-          // tS' = tQ K^T + Q tK^T
-          if (!mbar_wait(&full[sTK], ((ctr + 1) / C::NSLOT) & 1, abort_flag, p.status)) { ok = false; break; }
-          tc_fence_after();
+          ok = mbar_wait(&full[1], 0, abort_flag, p.status);
+          if (ok) {
+            tc_fence_after();
+            const uint32_t aTK = slot_addr(1);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            umma_ss(tmem + C::TM_TS, desc_kmajor(aTQ, C::BM, kk), desc_kmajor(aK, C::BN, kk),
-                    idesc_s, kk > 0);
+            for (int kk = 0; kk < D / 16; ++kk)
+              umma_ss(tmem + C::TM_TS, desc_kmajor(aTQ, C::BM, kk), desc_kmajor(aK, C::BN, kk),
+                      idesc_s, kk > 0);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            umma_ss(tmem + C::TM_TS, desc_kmajor(aQ, C::BM, kk), desc_kmajor(aTK, C::BN, kk),
-                    idesc_s, 1);
-          umma_commit(ts_full);
-          umma_commit(&empty[sK]);
-          umma_commit(&empty[sTK]);
-          if (idx == cnt - 1) umma_commit(q_empty);
-          // A += P V
-          if (!mbar_wait(p_full, p_ph, abort_flag, p.status)) { ok = false; break; }
+            for (int kk = 0; kk < D / 16; ++kk)
+              umma_ss(tmem + C::TM_TS, desc_kmajor(aQ, C::BM, kk), desc_kmajor(aTK, C::BN, kk),
+                      idesc_s, 1);
+            umma_commit(ts_full);
+            umma_commit(&empty[0]);
+            umma_commit(&empty[1]);
+            if (cnt == 1) umma_commit(q_empty);
+          }
+        }
+        while (ok) {
+          // the tile after g (same item or the next one)
+          bool has_next = true, new_item = false;
+          WorkItem w2 = w;
+          TileSched sch2 = sch;
+          int cnt2 = cnt, idx2 = idx + 1;
+          if (idx2 >= cnt) {
+            has_next = next_item(p, cta, G, k, pos);
+            if (has_next) {
+              ++k;
+              w2 = decode_item(p, pos);
+              sch2 = make_tile_sched(p.mask, w2.qt, C::BM, C::BN);
+              cnt2 = sch2.count();
+              idx2 = 0;
+              new_item = true;
+            }
+          }
+          const uint32_t c0 = 4 * g, c1 = 4 * (g + 1);
+          const uint32_t aTV = slot_addr(c0 + 2), aV = slot_addr(c0 + 3);
+          // T (+)= P tV, A (+)= P V
+          if (!mbar_wait(p_full, p_ph, abort_flag, p.status)) break;
           p_ph ^= 1;
-          tc_fence_after();
-          if (!mbar_wait(&full[sV], ((ctr + 2) / C::NSLOT) & 1, abort_flag, p.status)) { ok = false; break; }
+          if (!mbar_wait(&full[(c0 + 2) % C::NSLOT], slot_ph(c0 + 2), abort_flag, p.status)) break;
           tc_fence_after();
 #pragma unroll
           for (int ks = 0; ks < C::BN / 16; ++ks)
-            umma_ts(tmem + C::TM_A, tmem + C::TM_S + ks * 8, desc_mnmajor<C::BN>(aV, ks), idesc_v,
-                    (idx > 0 || ks > 0) ? 1u : 0u);
-          // T += U V + P tV
-          if (!mbar_wait(u_full, u_ph, abort_flag, p.status)) { ok = false; break; }
+            umma_ts(tmem + C::TM_T, tmem_a_operand(tmem + C::TM_S, ks), desc_mnmajor<C::BN>(aTV, ks),
+                    idesc_v, (idx > 0 || ks > 0) ? 1u : 0u);
+          umma_commit(&empty[(c0 + 2) % C::NSLOT]);
+          if (!mbar_wait(&full[(c0 + 3) % C::NSLOT], slot_ph(c0 + 3), abort_flag, p.status)) break;
+          tc_fence_after();
+#pragma unroll
+          for (int ks = 0; ks < C::BN / 16; ++ks)
+            umma_ts(tmem + C::TM_A, tmem_a_operand(tmem + C::TM_S, ks), desc_mnmajor<C::BN>(aV, ks),
+                    idesc_v, (idx > 0 || ks > 0) ? 1u : 0u);
+          // S_{g+1}
+          if (has_next) {
+            if (new_item) {
+              if (!mbar_wait(q_full, q_ph, abort_flag, p.status)) break;
+              q_ph ^= 1;
+            }
+            if (!mbar_wait(&full[c1 % C::NSLOT], slot_ph(c1), abort_flag, p.status)) break;
+            tc_fence_after();
+            const uint32_t aK = slot_addr(c1);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+              umma_ss(tmem + C::TM_S, desc_kmajor(aQ, C::BM, kk), desc_kmajor(aK, C::BN, kk), idesc_s,
+                      kk > 0);
+            umma_commit(s_full);
+          }
+          // T += U V
+          if (!mbar_wait(u_full, u_ph, abort_flag, p.status)) break;
           u_ph ^= 1;
           tc_fence_after();
-          if (!mbar_wait(&full[sTV], ((ctr + 3) / C::NSLOT) & 1, abort_flag, p.status)) { ok = false; break; }
-          tc_fence_after();
 #pragma unroll
           for (int ks = 0; ks < C::BN / 16; ++ks)
-            umma_ts(tmem + C::TM_T, tmem + C::TM_TS + ks * 8, desc_mnmajor<C::BN>(aV, ks), idesc_v,
-                    (idx > 0 || ks > 0) ? 1u : 0u);
-#pragma unroll
-          for (int ks = 0; ks < C::BN / 16; ++ks)
-            umma_ts(tmem + C::TM_T, tmem + C::TM_S + ks * 8, desc_mnmajor<C::BN>(aTV, ks), idesc_v, 1u);
-          umma_commit(&empty[sV]);
-          umma_commit(&empty[sTV]);
+            umma_ts(tmem + C::TM_T, tmem_a_operand(tmem + C::TM_TS, ks), desc_mnmajor<C::BN>(aV, ks),
+                    idesc_v, 1u);
+          umma_commit(&empty[(c0 + 3) % C::NSLOT]);
+          umma_commit(uv_done);
           if (idx == cnt - 1) umma_commit(acc_full);
+          if (!has_next) break;
+          // tS'_{g+1}
+          if (!mbar_wait(&full[(c1 + 1) % C::NSLOT], slot_ph(c1 + 1), abort_flag, p.status)) break;
+          tc_fence_after();
+          {
+            const uint32_t aK = slot_addr(c1), aTK = slot_addr(c1 + 1);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+              umma_ss(tmem + C::TM_TS, desc_kmajor(aTQ, C::BM, kk), desc_kmajor(aK, C::BN, kk),
+                      idesc_s, kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+              umma_ss(tmem + C::TM_TS, desc_kmajor(aQ, C::BM, kk), desc_kmajor(aTK, C::BN, kk),
+                      idesc_s, 1);
+          }
+          umma_commit(ts_full);
+          umma_commit(&empty[c1 % C::NSLOT]);
+          umma_commit(&empty[(c1 + 1) % C::NSLOT]);
+          if (idx2 == cnt2 - 1) umma_commit(q_empty);
+          w = w2;
+          sch = sch2;
+          cnt = cnt2;
+          idx = idx2;
+          ++g;
         }
       }
       // Every MMA issued so far completes before TMEM is released.
@@ -284,44 +383,78 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax + epilogue
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tS = tmem + lane_off + C::TM_S;
-    const uint32_t tTS = tmem + lane_off + C::TM_TS;
-    const uint32_t tA = tmem + lane_off + C::TM_A;
-    const uint32_t tT = tmem + lane_off + C::TM_T;
+    // Warpgroup wg (warps 4wg..4wg+3) owns key columns [64 wg, 64 wg + 64) of
+    // every score tile and output columns [D/2 wg, D/2 wg + D/2); thread
+    // (sub, lane) owns query row 32 sub + lane. The two warpgroups exchange
+    // their row maxima through shared memory each tile.
+    const int wg = warp >> 2, sub = warp & 3;
+    const int row = sub * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
+    const uint32_t tS = tmem + lane_off + C::TM_S + 64 * wg;
+    const uint32_t tTS = tmem + lane_off + C::TM_TS + 64 * wg;
+    const uint32_t tA = tmem + lane_off + C::TM_A + C::DH * wg;
+    const uint32_t tT = tmem + lane_off + C::TM_T + C::DH * wg;
+    float* my_x = xch + wg * C::BM + row;
+    const float* other_x = xch + (1 - wg) * C::BM + row;
+    uint32_t xa_ph = 0, xb_ph = 0;
+    // Swap one float per row with the other warpgroup (warps sub and sub + 4
+    // share rows): write, both arrive, read, both arrive. Bounded waits.
+    auto exchange = [&](float mine, float& theirs) -> bool {
+      *my_x = mine;
+      mbar_arrive(&xa[sub]);
+      if (!warp_wait(&xa[sub], xa_ph, abort_flag, p.status)) return false;
+      xa_ph ^= 1;
+      theirs = *other_x;
+      mbar_arrive(&xb[sub]);
+      if (!warp_wait(&xb[sub], xb_ph, abort_flag, p.status)) return false;
+      xb_ph ^= 1;
+      return true;
+    };
     const float scale_log2 = p.scale_log2;
     const float scale = p.scale;
-    uint32_t s_ph = 0, ts_ph = 0, acc_ph = 0;
+    uint32_t s_ph = 0, ts_ph = 0, acc_ph = 0, g = 0;
     bool ok = true;
-    for (int k = 0; ok && k * G < p.n_items; ++k) {
-      const int pos = item_position(k, cta, G);
-      if (pos >= p.n_items) continue;
+    int k = 0, pos = 0;
+    while (ok && next_item(p, cta, G, k, pos)) {
+      ++k;
       const WorkItem w = decode_item(p, pos);
-      const int t = w.qt * C::BM + warp * 32 + lane;  // this thread's query row
+      const int t = w.qt * C::BM + row;  // this thread's query row
       const RowRange rr = row_range(p.mask, t);
       const TileSched sch = make_tile_sched(p.mask, w.qt, C::BM, C::BN);
       const int cnt = sch.count();
       float m_use = -INFINITY, l = 0.f, dsum = 0.f;
-      for (int idx = 0; idx < cnt; ++idx) {
+      for (int idx = 0; idx < cnt; ++idx, ++g) {
         const int kt = sch.tile(idx);
         const bool full_tile = sch.full(kt);
-        const int k0 = kt * C::BN;
+        const int k0 = kt * C::BN + C::HALF * wg;
         if (!warp_wait(s_full, s_ph, abort_flag, p.status)) { ok = false; break; }
         s_ph ^= 1;
         tc_fence_after();
-        uint32_t sr[C::BN];
-#pragma unroll
-        for (int c = 0; c < C::BN / 32; ++c)
-          tmem_ld32(tS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
+        uint32_t sr[C::HALF];
+        tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
         tmem_wait_ld();
-        float x[C::BN];
-        float mt = -INFINITY;
+        if (!full_tile) {
 #pragma unroll
-        for (int j = 0; j < C::BN; ++j) {
-          x[j] = __uint_as_float(sr[j]) * scale_log2;
-          if (!full_tile && !row_allows(rr, k0 + j)) x[j] = -INFINITY;
-          mt = fmaxf(mt, x[j]);
+          for (int j = 0; j < C::HALF; ++j)
+            if (!row_allows(rr, k0 + j)) sr[j] = __float_as_uint(-INFINITY);
         }
+        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < C::HALF; j += 4) {
+          mx0 = fmaxf(mx0, __uint_as_float(sr[j]));
+          mx1 = fmaxf(mx1, __uint_as_float(sr[j + 1]));
+          mx2 = fmaxf(mx2, __uint_as_float(sr[j + 2]));
+          mx3 = fmaxf(mx3, __uint_as_float(sr[j + 3]));
+        }
+        const float my_max = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        // row maximum over both halves of the tile
+        float their_max;
+        tc_fence_before();
+        if (!exchange(my_max, their_max)) { ok = false; break; }
+        tc_fence_after();
+        const float row_max = fmaxf(my_max, their_max);
+        const float mt = row_max * scale_log2;  // log2 units; -inf if fully masked
         bool resc = false;
         float alpha = 1.f;
         if (m_use == -INFINITY) {
@@ -334,37 +467,47 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
           resc = true;
         }
         if (__any_sync(0xffffffffu, resc)) {
-          // All value MMAs of earlier tiles are complete (S of this tile was
-          // issued after them), so A and T can be rescaled in place.
+          // A: every P V of earlier tiles is complete (S of this tile was
+          // issued after it). T: wait for the U V of the previous tile.
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t a[32], tt[32];
+          for (int c = 0; c < C::DH / 32; ++c) {
+            uint32_t a[32];
             tmem_ld32(tA + 32 * c, a);
-            tmem_ld32(tT + 32 * c, tt);
             tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              a[j] = __float_as_uint(__uint_as_float(a[j]) * alpha);
-              tt[j] = __float_as_uint(__uint_as_float(tt[j]) * alpha);
-            }
+            for (int j = 0; j < 32; ++j) a[j] = __float_as_uint(__uint_as_float(a[j]) * alpha);
             tmem_st32(tA + 32 * c, a);
-            tmem_st32(tT + 32 * c, tt);
+          }
+          if (!warp_wait(uv_done, (g - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < C::DH / 32; ++c) {
+            uint32_t a[32];
+            tmem_ld32(tT + 32 * c, a);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) a[j] = __float_as_uint(__uint_as_float(a[j]) * alpha);
+            tmem_st32(tT + 32 * c, a);
           }
         }
         const float mb = (m_use == -INFINITY) ? 0.f : m_use;
-        uint32_t pk[C::BN / 2];
-        float lsum = 0.f;
+        uint32_t pk[C::HALF / 2];
+        float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
 #pragma unroll
-        for (int j = 0; j < C::BN / 2; ++j) {
-          const float p0 = ex2_approx(x[2 * j] - mb);
-          const float p1 = ex2_approx(x[2 * j + 1] - mb);
-          lsum += p0 + p1;
+        for (int j = 0; j < C::HALF / 2; j += 2) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * j]), scale_log2, -mb));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * j + 1]), scale_log2, -mb));
+          const float p2 = ex2_approx(fmaf(__uint_as_float(sr[2 * j + 2]), scale_log2, -mb));
+          const float p3 = ex2_approx(fmaf(__uint_as_float(sr[2 * j + 3]), scale_log2, -mb));
+          ls0 += p0;
+          ls1 += p1;
+          ls2 += p2;
+          ls3 += p3;
           pk[j] = pack_bf16x2(p0, p1);
+          pk[j + 1] = pack_bf16x2(p2, p3);
         }
-        l += lsum;
-#pragma unroll
-        for (int c = 0; c < C::BN / 64; ++c)
-          tmem_st32(tS + 32 * c, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32 * c]));
+        l += (ls0 + ls1) + (ls2 + ls3);
+        tmem_st32(tS, pk);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -373,24 +516,31 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
         if (!warp_wait(ts_full, ts_ph, abort_flag, p.status)) { ok = false; break; }
         ts_ph ^= 1;
         tc_fence_after();
-        float ds = 0.f;
+        uint32_t v[C::HALF];
+        tmem_ld32(tTS, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld32(tTS + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        tmem_wait_ld();
+        uint32_t uk[C::HALF / 2];
+        float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
 #pragma unroll
-        for (int c = 0; c < C::BN / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tTS + 32 * c, v);
-          tmem_wait_ld();
-          uint32_t uk[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const uint32_t pp = pk[16 * c + j];
-            const float u0 = bf16lo_to_f32(pp) * scale * __uint_as_float(v[2 * j]);
-            const float u1 = bf16hi_to_f32(pp) * scale * __uint_as_float(v[2 * j + 1]);
-            ds += u0 + u1;
-            uk[j] = pack_bf16x2(u0, u1);
-          }
-          tmem_st16(tTS + 16 * c, uk);
+        for (int j = 0; j < C::HALF / 2; j += 2) {
+          const float q0 = bf16lo_to_f32(pk[j]) * scale;
+          const float q1 = bf16hi_to_f32(pk[j]) * scale;
+          const float q2 = bf16lo_to_f32(pk[j + 1]) * scale;
+          const float q3 = bf16hi_to_f32(pk[j + 1]) * scale;
+          const float u0 = q0 * __uint_as_float(v[2 * j]);
+          const float u1 = q1 * __uint_as_float(v[2 * j + 1]);
+          const float u2 = q2 * __uint_as_float(v[2 * j + 2]);
+          const float u3 = q3 * __uint_as_float(v[2 * j + 3]);
+          d0 += u0;
+          d1 += u1;
+          d2 += u2;
+          d3 += u3;
+          uk[j] = pack_bf16x2(u0, u1);
+          uk[j + 1] = pack_bf16x2(u2, u3);
         }
-        dsum += ds;
+        dsum += (d0 + d1) + (d2 + d3);
+        tmem_st32(tTS, uk);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -401,14 +551,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
       if (!warp_wait(acc_full, acc_ph, abort_flag, p.status)) { ok = false; break; }
       acc_ph ^= 1;
       tc_fence_after();
+      float l_other, d_other;
+      if (!exchange(l, l_other) || !exchange(dsum, d_other)) { ok = false; break; }
+      const float l_tot = l + l_other;
+      const float d_tot = dsum + d_other;
       const bool valid = t < p.L;
-      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-      const float mu = dsum * inv_l;
-      const size_t row_off = ((static_cast<size_t>(w.b) * p.L + (valid ? t : 0)) * p.H + w.h) * D;
+      const float inv_l = (l_tot > 0.f) ? 1.f / l_tot : 0.f;
+      const float mu = d_tot * inv_l;
+      const size_t row_off =
+          ((static_cast<size_t>(w.b) * p.L + (valid ? t : 0)) * p.H + w.h) * D + C::DH * wg;
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + row_off;
       __nv_bfloat16* torow = reinterpret_cast<__nv_bfloat16*>(p.to) + row_off;
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < C::DH / 32; ++c) {
         uint32_t a[32], tt[32];
         tmem_ld32(tA + 32 * c, a);
         tmem_ld32(tT + 32 * c, tt);
@@ -433,9 +588,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
           }
         }
       }
-      if (valid) {
+      if (valid && wg == 0) {
         const float mb = (m_use == -INFINITY) ? 0.f : m_use;
-        p.lse[(static_cast<size_t>(w.b) * p.H + w.h) * p.L + t] = (mb + __log2f(l)) * kLn2;
+        p.lse[(static_cast<size_t>(w.b) * p.H + w.h) * p.L + t] = (mb + __log2f(l_tot)) * kLn2;
       }
     }
     tc_fence_before();
@@ -443,7 +598,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
 
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) tmem_dealloc(tmem, C::TM_COLS);
+  if (warp == 9) tmem_dealloc(tmem, C::TM_COLS);
 }
 
 size_t tc_smem_bytes(int d) { return d == 128 ? TcCfg<128>::BYTES : TcCfg<64>::BYTES; }

@@ -12,7 +12,7 @@ namespace ajvp {
 // ---- bf16 tensor-core kernel (tcgen05 / TMEM / TMA) ----
 constexpr int kTcBlockM = 128;   // query rows per tile (one TMEM lane per row)
 constexpr int kTcBlockN = 128;   // keys per tile
-constexpr int kTcThreads = 192;  // warps 0-3 softmax+epilogue, 4 TMA producer, 5 MMA issuer
+constexpr int kTcThreads = 320;  // warps 0-7 softmax+epilogue, 8 TMA producer, 9 MMA issuer
 constexpr int kMaxOrder = 4096;  // longest-first query-tile order table capacity
 
 struct TcParams {

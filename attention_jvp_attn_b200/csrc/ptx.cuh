@@ -228,6 +228,11 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
 }
 
+// Named barrier over `nthreads` threads (a multiple of 32) of this CTA.
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // ---------------------------------------------------------------- math
 // Hardware base-2 exponential (MUFU.EX2), flushing denormals; exp2(-inf) = 0.
 __device__ __forceinline__ float ex2_approx(float x) {

@@ -124,11 +124,12 @@ def make_inputs(w: Workload, device="cpu", seed: Optional[int] = None,
 
 
 def sample_rows(w: Workload, n_random: int = 256, seed: int = 7,
-                tile: int = 128) -> List[int]:
+                tile: int = 128, max_rows: Optional[int] = None) -> List[int]:
     """Query rows worth checking one by one on a large workload: first and
     last row of every chunk (clean and noisy), the rows on both sides of the
     `tile` boundaries around every chunk boundary (where tiles are partial),
-    the ragged tail, and `n_random` seeded random rows."""
+    the ragged tail, and `n_random` seeded random rows. With `max_rows`, a
+    seeded subset of that size (always keeping the first and last row)."""
     L, c = w.L, w.chunk_tokens
     rows = set()
     for j in range(L // c):
@@ -140,4 +141,8 @@ def sample_rows(w: Workload, n_random: int = 256, seed: int = 7,
     rows.update((L - 1, (L - 1) // tile * tile, (L - 1) // tile * tile - 1))
     g = torch.Generator().manual_seed(seed)
     rows.update(torch.randint(0, L, (n_random,), generator=g).tolist())
-    return sorted(r for r in rows if 0 <= r < L)
+    out = sorted(r for r in rows if 0 <= r < L)
+    if max_rows is not None and len(out) > max_rows:
+        keep = torch.randperm(len(out), generator=g)[:max_rows - 2].tolist()
+        out = sorted({out[0], out[-1], *(out[i] for i in keep)})
+    return out

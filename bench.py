@@ -136,11 +136,14 @@ class ClockSampler:
                 "power_w_max": max(power) if power else None}
 
 
-def workload_by_name(name):
+def workload_by_name(name, heads=None):
     from attention_jvp_attn_b200 import inputs as wl
     if name not in wl.WORKLOADS:
         raise SystemExit(f"unknown workload {name}; choose from {sorted(wl.WORKLOADS)}")
-    return wl.WORKLOADS[name]
+    w = wl.WORKLOADS[name]
+    if heads is not None:
+        w = w.with_(H=heads, name=f"{w.name}_h{heads}")
+    return w
 
 
 def flops_per_step(w) -> int:
@@ -201,7 +204,7 @@ def run_reference(args):
     world = _env_int("WORLD_SIZE", 1)
     if rank != 0:
         return 0
-    w = workload_by_name(args.workload)
+    w = workload_by_name(args.workload, args.heads)
     for _ in range(args.warmup):
         oracle_sample(w, budget_s=0.5)
     vals, secs, rows_all = [], 0.0, 0
@@ -254,7 +257,7 @@ def run_gpu(args):
         if world > 1:
             dist.barrier()
 
-    w = workload_by_name(args.workload)
+    w = workload_by_name(args.workload, args.heads)
     x = wl.make_inputs(w, device=dev, seed=w.seed + 7919 * rank)
     B, L, H, d = w.B, w.L, w.H, w.d
     dt = x["q"].dtype
@@ -378,6 +381,7 @@ def main():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="framewise_tf_bf16")
+    ap.add_argument("--heads", type=int, default=None, help="override H (profiling a smaller case)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")

@@ -90,10 +90,10 @@ def test_small_custom_scale_and_distributions(cuda_device):
     _dense_check(w, cuda_device)
 
 
-def _sampled_check(w, device, heads=(0, -1), n_random=256):
+def _sampled_check(w, device, heads=(0, -1), n_random=256, max_rows=None):
     x = wl.make_inputs(w, device=device)
     o, to, lse = _run(w, x)
-    rows = wl.sample_rows(w, n_random=n_random)
+    rows = wl.sample_rows(w, n_random=n_random, max_rows=max_rows)
     t_o, t_l = TOL[w.dtype]
     worst = 0.0
     for b in sorted({0, w.B - 1}):
@@ -118,7 +118,7 @@ def test_full_size_sampled_rows(cuda_device, w):
 
 @pytest.mark.parametrize("w", wl.sweep_points(), ids=lambda w: w.name)
 def test_sweep_sampled_rows(cuda_device, w):
-    _sampled_check(w, cuda_device, heads=(5,), n_random=32)
+    _sampled_check(w, cuda_device, heads=(5,), n_random=32, max_rows=256)
 
 
 def test_deterministic(cuda_device):

@@ -35,17 +35,19 @@ _lib = None
 _lock = threading.Lock()
 
 
-def load() -> ctypes.CDLL:
-    """Load the in-tree CUDA library; raise if it has not been built."""
+def load(path: str = None) -> ctypes.CDLL:
+    """Load the in-tree CUDA library (or the library at `path`, e.g. the trace
+    build, which then serves every later call); raise if it is missing."""
     global _lib
     with _lock:
-        if _lib is not None:
+        if _lib is not None and path is None:
             return _lib
-        if not os.path.exists(LIB_PATH):
+        path = path or os.environ.get("ATTN_JVP_LIB", LIB_PATH)
+        if not os.path.exists(path):
             raise RuntimeError(
-                f"CUDA library not built: {LIB_PATH} is missing "
+                f"CUDA library not built: {path} is missing "
                 "(run `python -m attention_jvp_attn_b200.build`)")
-        lib = ctypes.CDLL(LIB_PATH)
+        lib = ctypes.CDLL(path)
         vp = ctypes.c_void_p
         lib.attn_jvp_fwd.argtypes = [ctypes.POINTER(Shape), vp, vp, vp, vp, vp, vp, Mask,
                                      vp, vp, vp, vp]

@@ -19,6 +19,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libattn_jvp.so")
+# Opt-in variant whose bf16 kernel records per-tile event clocks of CTA 0.
+TRACE_LIB = os.path.join(PKG, "libattn_jvp_trace.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -38,19 +40,21 @@ def _deps():
     return _sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h"))
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(f) <= t for f in _deps())
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
+def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False,
+          trace: bool = False) -> str:
+    lib = TRACE_LIB if trace else LIB
+    if not force and up_to_date(lib):
+        return lib
     cmd = [_nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr",
            "-Xcompiler", "-fPIC,-O2", "-shared", "-I", INCLUDE, "-I", CSRC,
-           "-o", LIB + ".tmp", *_sources()]
+           *(["-DAJVP_TRACE"] if trace else []), "-o", lib + ".tmp", *_sources()]
     if ptxas_info:
         cmd[1:1] = ["-Xptxas", "-v"]
     if verbose:
@@ -60,11 +64,10 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
         raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stdout}\n{res.stderr}")
     if verbose or ptxas_info:
         sys.stdout.write(res.stdout + res.stderr)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(lib + ".tmp", lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="--verbose" in sys.argv,
-          ptxas_info="--ptxas-info" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv,
+                ptxas_info="--ptxas-info" in sys.argv, trace="--trace" in sys.argv))

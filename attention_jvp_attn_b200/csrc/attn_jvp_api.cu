@@ -36,6 +36,9 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn g_encode = nullptr;
+#ifdef AJVP_TRACE
+long long* g_trace = nullptr;
+#endif
 
 // Per-device set-up, done once under the lock: checks the device is sm_100,
 // allocates the 4-byte status word and raises the kernels' shared-memory limit.
@@ -182,6 +185,9 @@ int launch_bf16(DeviceState* st, const attn_jvp_shape* s, const void* q, const v
   p.scale = sc;
   p.scale_log2 = sc * 1.4426950408889634f;
   p.order_len = fill_order(p.mask, p.n_qtiles, p.order);
+#ifdef AJVP_TRACE
+  p.trace = g_trace;
+#endif
   const int grid = std::min(st->sm_count, p.n_items);
   if (ajvp::tc_launch(static_cast<int>(s->d), p, grid, stream) != cudaSuccess)
     return ATTN_JVP_ERR_CUDA;
@@ -339,5 +345,11 @@ int32_t attn_jvp_schedule_tiles(attn_jvp_mask mask, int64_t L, int32_t block_m, 
 }
 
 int32_t attn_jvp_version(void) { return 100; }
+
+#ifdef AJVP_TRACE
+// Trace builds only: device buffer of kTraceTiles x kTraceEvents int64 clocks
+// that the next bf16 launches fill for CTA 0 (NULL disables).
+void attn_jvp_set_trace(void* dev_buf) { g_trace = static_cast<long long*>(dev_buf); }
+#endif
 
 }  // extern "C"

@@ -41,6 +41,34 @@ namespace ajvp {
 constexpr float kRescaleTau = 8.0f;
 constexpr float kLn2 = 0.69314718055994530942f;
 
+// Event clocks of CTA kTraceCta for its first kTraceTiles key tiles (trace builds only).
+#ifdef AJVP_TRACE
+#define AJVP_EV(tile, ev)                                                             \
+  do {                                                                                \
+    if (p.trace && blockIdx.x == kTraceCta && (tile) < kTraceTiles)                   \
+      p.trace[(tile) * kTraceEvents + (ev)] = static_cast<long long>(clock64());      \
+  } while (0)
+// Clock read issued after the register holding x is available.
+__device__ __forceinline__ long long clock_after(float x) {
+  long long t;
+  asm volatile("{\n\t.reg .pred q;\n\tsetp.eq.f32 q, %1, 0f46404C00;\n\tmov.u64 %0, %%clock64;\n\t}"
+               : "=l"(t) : "f"(x));
+  return t;
+}
+#define AJVP_EVX(tile, ev, val)                                                      \
+  do {                                                                               \
+    if (p.trace && blockIdx.x == kTraceCta && (tile) < kTraceTiles)                  \
+      p.trace[(tile) * kTraceEvents + (ev)] = clock_after(val);                      \
+  } while (0)
+#else
+#define AJVP_EVX(tile, ev, val) \
+  do {                          \
+  } while (0)
+#define AJVP_EV(tile, ev) \
+  do {                    \
+  } while (0)
+#endif
+
 template <int D>
 struct TcCfg {
   static constexpr int BM = kTcBlockM;
@@ -86,6 +114,11 @@ __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t base, int ks) {
 // [16 ks, 16 ks + 16).
 __device__ __forceinline__ uint32_t tmem_a_operand(uint32_t base, int ks) {
   return base + 64 * (ks >> 2) + (ks & 3) * 8;
+}
+
+// Bit mask of the lowest n bits (n clamped to [0, 32]).
+__device__ __forceinline__ uint32_t low_bits(int n) {
+  return n <= 0 ? 0u : (n >= 32 ? 0xffffffffu : ((1u << n) - 1u));
 }
 
 struct WorkItem {
@@ -309,8 +342,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
           const uint32_t c0 = 4 * g, c1 = 4 * (g + 1);
           const uint32_t aTV = slot_addr(c0 + 2), aV = slot_addr(c0 + 3);
           // T (+)= P tV, A (+)= P V
+          AJVP_EV(g, 0);
           if (!mbar_wait(p_full, p_ph, abort_flag, p.status)) break;
           p_ph ^= 1;
+          AJVP_EV(g, 1);
           if (!mbar_wait(&full[(c0 + 2) % C::NSLOT], slot_ph(c0 + 2), abort_flag, p.status)) break;
           tc_fence_after();
 #pragma unroll
@@ -338,10 +373,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
               umma_ss(tmem + C::TM_S, desc_kmajor(aQ, C::BM, kk), desc_kmajor(aK, C::BN, kk), idesc_s,
                       kk > 0);
             umma_commit(s_full);
+            AJVP_EV(g, 2);
           }
           // T += U V
           if (!mbar_wait(u_full, u_ph, abort_flag, p.status)) break;
           u_ph ^= 1;
+          AJVP_EV(g, 3);
           tc_fence_after();
 #pragma unroll
           for (int ks = 0; ks < C::BN / 16; ++ks)
@@ -366,6 +403,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
                       idesc_s, 1);
           }
           umma_commit(ts_full);
+          AJVP_EV(g, 4);
           umma_commit(&empty[c1 % C::NSLOT]);
           umma_commit(&empty[(c1 + 1) % C::NSLOT]);
           if (idx2 == cnt2 - 1) umma_commit(q_empty);
@@ -429,15 +467,25 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
         const int k0 = kt * C::BN + C::HALF * wg;
         if (!warp_wait(s_full, s_ph, abort_flag, p.status)) { ok = false; break; }
         s_ph ^= 1;
+        if (warp == 0 && lane == 0) AJVP_EV(g, 5);
         tc_fence_after();
         uint32_t sr[C::HALF];
         tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
         tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
         tmem_wait_ld();
         if (!full_tile) {
+          // admissible local columns of this row in this half tile, [0, e1) U
+          // [s2, e2), as 32-bit column masks
+          const int e1 = min(max(rr.a1 - k0, 0), C::HALF);
+          const int s2 = min(max(rr.b0 - k0, 0), C::HALF);
+          const int e2 = min(max(rr.b1 - k0, 0), C::HALF);
 #pragma unroll
-          for (int j = 0; j < C::HALF; ++j)
-            if (!row_allows(rr, k0 + j)) sr[j] = __float_as_uint(-INFINITY);
+          for (int q = 0; q < C::HALF / 32; ++q) {
+            const uint32_t m = low_bits(e1 - 32 * q) | (low_bits(e2 - 32 * q) & ~low_bits(s2 - 32 * q));
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (!((m >> j) & 1u)) sr[32 * q + j] = __float_as_uint(-INFINITY);
+          }
         }
         float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
@@ -454,6 +502,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
         if (!exchange(my_max, their_max)) { ok = false; break; }
         tc_fence_after();
         const float row_max = fmaxf(my_max, their_max);
+        if (warp == 0 && lane == 0) AJVP_EV(g, 6);
         const float mt = row_max * scale_log2;  // log2 units; -inf if fully masked
         bool resc = false;
         float alpha = 1.f;
@@ -512,9 +561,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(p_full);
+        if (warp == 0 && lane == 0) AJVP_EV(g, 7);
 
         if (!warp_wait(ts_full, ts_ph, abort_flag, p.status)) { ok = false; break; }
         ts_ph ^= 1;
+        if (warp == 0 && lane == 0) AJVP_EV(g, 8);
         tc_fence_after();
         uint32_t v[C::HALF];
         tmem_ld32(tTS, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
@@ -545,6 +596,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(u_full);
+        if (warp == 0 && lane == 0) AJVP_EV(g, 9);
       }
       if (!ok) break;
       // ---------------- epilogue: O = A/l, tO = T/l - (D/l) O, LSE

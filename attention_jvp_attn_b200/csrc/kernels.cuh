@@ -28,8 +28,17 @@ struct TcParams {
   float scale_log2;  // s * log2(e)
   float scale;       // s
   int order_len;     // n_qtiles if `order` is filled, else 0 (reverse index order)
+#ifdef AJVP_TRACE
+  long long* trace;  // per-tile event clocks of CTA 0 (trace builds only)
+#endif
   uint16_t order[kMaxOrder];
 };
+
+#ifdef AJVP_TRACE
+constexpr int kTraceTiles = 512;
+constexpr int kTraceEvents = 16;
+constexpr int kTraceCta = 5;  // a CTA whose first items are mostly full tiles
+#endif
 
 size_t tc_smem_bytes(int d);
 cudaError_t tc_prepare(int d);  // sets the dynamic shared-memory limit (once per device)

@@ -92,21 +92,12 @@ struct TcCfg {
   static_assert(TM_T + D <= TM_COLS, "TMEM budget");
 };
 
-// K-major operand (rows of 64-element / 128-byte swizzled chunks, chunk c of
-// a `rows`-row tile at c * rows * 128 bytes): k-step kk covers elements
-// [16 kk, 16 kk + 16) of the contraction dimension.
-__device__ __forceinline__ uint64_t desc_kmajor(uint32_t base, int rows, int kk) {
-  const uint32_t addr = base + (kk >> 2) * rows * 128 + (kk & 3) * 32;
-  return smem_desc_sw128(addr, 16, 1024);
-}
-
-// MN-major operand: a V tile [BN keys x D] read as B[K = keys, N = d]; k-step
-// ks covers keys [16 ks, 16 ks + 16). 64-element N blocks sit BN*128 bytes
-// apart (LBO), 8-key groups 1024 bytes apart (SBO).
-template <int BN>
-__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t base, int ks) {
-  return smem_desc_sw128(base + ks * 16 * 128, BN * 128, 1024);
-}
+// Operand layouts in shared memory (TMA, 128-byte swizzle): a tile of R rows
+// x D columns is D/64 chunks of R rows x 128 bytes. As a K-major operand
+// (Q, tQ, K, tK: contraction over d) k-step kk starts at chunk kk/4, byte
+// 32 (kk%4); the stride between 8-row groups (SBO) is 1024. As an MN-major
+// operand (V, tV: contraction over keys) k-step ks starts at key 16 ks; the
+// 64-column blocks of d sit R*128 bytes apart (LBO), 8-key groups 1024.
 
 // bf16 P (or U) in TMEM: warpgroup h packs keys [64 h, 64 h + 64) into the
 // first 32 of its own 64 score columns, so key k sits at column
@@ -114,6 +105,34 @@ __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t base, int ks) {
 // [16 ks, 16 ks + 16).
 __device__ __forceinline__ uint32_t tmem_a_operand(uint32_t base, int ks) {
   return base + 64 * (ks >> 2) + (ks & 3) * 8;
+}
+
+// Score MMA: D[tmem] (+)= A B^T over the head dimension, A a [rows_a x D]
+// and B a [rows_b x D] K-major tile. Offsets are added to the descriptors'
+// start-address field (16-byte units; tiles lie well inside its 256 KB range).
+template <int D, int ROWS_A, int ROWS_B>
+__device__ __forceinline__ void mma_scores(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem,
+                                           uint32_t idesc, bool accumulate) {
+  const uint64_t da = smem_desc_sw128(a_smem, 16, 1024);
+  const uint64_t db = smem_desc_sw128(b_smem, 16, 1024);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t oa = ((kk >> 2) * ROWS_A * 128 + (kk & 3) * 32) >> 4;
+    const uint32_t ob = ((kk >> 2) * ROWS_B * 128 + (kk & 3) * 32) >> 4;
+    umma_ss(d_tmem, da + oa, db + ob, idesc, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+// Value MMA: D[tmem] (+)= P[tmem] V, P a bf16 [128 x BN] tile in TMEM (in the
+// two-warpgroup layout of tmem_a_operand) and V a [BN keys x D] tile read MN-major.
+template <int BN>
+__device__ __forceinline__ void mma_values_split(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem,
+                                           uint32_t idesc, bool accumulate) {
+  const uint64_t db = smem_desc_sw128(b_smem, BN * 128, 1024);
+#pragma unroll
+  for (int ks = 0; ks < BN / 16; ++ks)
+    umma_ts(d_tmem, tmem_a_operand(a_tmem, ks), db + ((ks * 16 * 128) >> 4), idesc,
+            (accumulate || ks > 0) ? 1u : 0u);
 }
 
 // Bit mask of the lowest n bits (n clamped to [0, 32]).
@@ -299,23 +318,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
         if (ok) {
           tc_fence_after();
           const uint32_t aK = slot_addr(0);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            umma_ss(tmem + C::TM_S, desc_kmajor(aQ, C::BM, kk), desc_kmajor(aK, C::BN, kk), idesc_s,
-                    kk > 0);
+mma_scores<D, C::BM, C::BN>(tmem + C::TM_S, aQ, aK, idesc_s, false);
           umma_commit(s_full);
           ok = mbar_wait(&full[1], 0, abort_flag, p.status);
           if (ok) {
             tc_fence_after();
             const uint32_t aTK = slot_addr(1);
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk)
-              umma_ss(tmem + C::TM_TS, desc_kmajor(aTQ, C::BM, kk), desc_kmajor(aK, C::BN, kk),
-                      idesc_s, kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk)
-              umma_ss(tmem + C::TM_TS, desc_kmajor(aQ, C::BM, kk), desc_kmajor(aTK, C::BN, kk),
-                      idesc_s, 1);
+mma_scores<D, C::BM, C::BN>(tmem + C::TM_TS, aTQ, aK, idesc_s, false);
+mma_scores<D, C::BM, C::BN>(tmem + C::TM_TS, aQ, aTK, idesc_s, true);
             umma_commit(ts_full);
             umma_commit(&empty[0]);
             umma_commit(&empty[1]);
@@ -348,17 +358,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
           AJVP_EV(g, 1);
           if (!mbar_wait(&full[(c0 + 2) % C::NSLOT], slot_ph(c0 + 2), abort_flag, p.status)) break;
           tc_fence_after();
-#pragma unroll
-          for (int ks = 0; ks < C::BN / 16; ++ks)
-            umma_ts(tmem + C::TM_T, tmem_a_operand(tmem + C::TM_S, ks), desc_mnmajor<C::BN>(aTV, ks),
-                    idesc_v, (idx > 0 || ks > 0) ? 1u : 0u);
+mma_values_split<C::BN>(tmem + C::TM_T, tmem + C::TM_S, aTV, idesc_v, idx > 0);
           umma_commit(&empty[(c0 + 2) % C::NSLOT]);
           if (!mbar_wait(&full[(c0 + 3) % C::NSLOT], slot_ph(c0 + 3), abort_flag, p.status)) break;
           tc_fence_after();
-#pragma unroll
-          for (int ks = 0; ks < C::BN / 16; ++ks)
-            umma_ts(tmem + C::TM_A, tmem_a_operand(tmem + C::TM_S, ks), desc_mnmajor<C::BN>(aV, ks),
-                    idesc_v, (idx > 0 || ks > 0) ? 1u : 0u);
+mma_values_split<C::BN>(tmem + C::TM_A, tmem + C::TM_S, aV, idesc_v, idx > 0);
           // S_{g+1}
           if (has_next) {
             if (new_item) {
@@ -368,10 +372,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
             if (!mbar_wait(&full[c1 % C::NSLOT], slot_ph(c1), abort_flag, p.status)) break;
             tc_fence_after();
             const uint32_t aK = slot_addr(c1);
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk)
-              umma_ss(tmem + C::TM_S, desc_kmajor(aQ, C::BM, kk), desc_kmajor(aK, C::BN, kk), idesc_s,
-                      kk > 0);
+mma_scores<D, C::BM, C::BN>(tmem + C::TM_S, aQ, aK, idesc_s, false);
             umma_commit(s_full);
             AJVP_EV(g, 2);
           }
@@ -380,10 +381,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
           u_ph ^= 1;
           AJVP_EV(g, 3);
           tc_fence_after();
-#pragma unroll
-          for (int ks = 0; ks < C::BN / 16; ++ks)
-            umma_ts(tmem + C::TM_T, tmem_a_operand(tmem + C::TM_TS, ks), desc_mnmajor<C::BN>(aV, ks),
-                    idesc_v, 1u);
+mma_values_split<C::BN>(tmem + C::TM_T, tmem + C::TM_TS, aV, idesc_v, true);
           umma_commit(&empty[(c0 + 3) % C::NSLOT]);
           umma_commit(uv_done);
           if (idx == cnt - 1) umma_commit(acc_full);
@@ -393,14 +391,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
           tc_fence_after();
           {
             const uint32_t aK = slot_addr(c1), aTK = slot_addr(c1 + 1);
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk)
-              umma_ss(tmem + C::TM_TS, desc_kmajor(aTQ, C::BM, kk), desc_kmajor(aK, C::BN, kk),
-                      idesc_s, kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk)
-              umma_ss(tmem + C::TM_TS, desc_kmajor(aQ, C::BM, kk), desc_kmajor(aTK, C::BN, kk),
-                      idesc_s, 1);
+mma_scores<D, C::BM, C::BN>(tmem + C::TM_TS, aTQ, aK, idesc_s, false);
+mma_scores<D, C::BM, C::BN>(tmem + C::TM_TS, aQ, aTK, idesc_s, true);
           }
           umma_commit(ts_full);
           AJVP_EV(g, 4);

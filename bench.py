@@ -31,6 +31,29 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+METRIC = "attention+JVP effective TFLOP/s (unmasked pairs) and % of B200 bf16 peak"
+RANK_SEED_STRIDE = 7919
+
+
+def rank_seed(w, rank: int) -> int:
+    """Seed of a rank's replica of the workload (replicas draw different inputs)."""
+    return w.seed + RANK_SEED_STRIDE * rank
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """Maximum of a per-rank timing over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, flops_per_step: int, steps: int, max_ms: float) -> float:
+    """Whole-job TFLOP/s: every rank ran `steps` steps; time is the slowest rank's."""
+    return world * flops_per_step * steps / (max_ms * 1e-3) / 1e12
 
 
 def _env_int(name, default):
@@ -231,7 +254,6 @@ def run_reference(args):
     return 0
 
 
-METRIC = "attention+JVP effective TFLOP/s (unmasked pairs) and % of B200 bf16 peak"
 
 
 # --------------------------------------------------------------------------- GPU arm
@@ -258,7 +280,7 @@ def run_gpu(args):
             dist.barrier()
 
     w = workload_by_name(args.workload, args.heads)
-    x = wl.make_inputs(w, device=dev, seed=w.seed + 7919 * rank)
+    x = wl.make_inputs(w, device=dev, seed=rank_seed(w, rank))
     B, L, H, d = w.B, w.L, w.H, w.d
     dt = x["q"].dtype
     o = torch.empty_like(x["q"])
@@ -299,13 +321,10 @@ def run_gpu(args):
         raise SystemExit(f"device status {st} after timed steps")
     total_ms = t_begin.elapsed_time(t_end)
     launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    if world > 1:
-        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(total_ms, dev)
     ms_per_step = total_ms / args.steps
     flops = flops_per_step(w)
-    value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
+    value = job_throughput(world, flops, args.steps, total_ms)
 
     # end to end through the host-buffer C-ABI entry point (pinned host memory)
     e2e = None
@@ -329,13 +348,9 @@ def run_gpu(args):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        e2e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e2e_ms = float(tt.item())
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
         tensor_bytes = B * L * H * d * x["q"].element_size()
-        e2e = {"value": world * flops * args.e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": job_throughput(world, flops, args.e2e_steps, e2e_ms), "unit": "TFLOP/s",
                "ms_per_step": e2e_ms / args.e2e_steps,
                "h2d_bytes_per_step": 6 * tensor_bytes,
                "d2h_bytes_per_step": 2 * tensor_bytes + B * H * L * 4}

@@ -84,10 +84,50 @@ def test_small_dense(cuda_device, dtype, mode, c, n, d, B, H):
     _dense_check(w, cuda_device)
 
 
+def _rounding_bound(x, w):
+    """First-order error bound of the bf16 path, per output element, from the
+    bf16 rounding (unit 2^-9) of P and U = P s tS before their tensor-core
+    products and of the outputs: for O, 2^-9 (sum_j P|v| + |O|); for tO,
+    2^-9 (2 sum_j P|tS||v| + sum_j P|tv| + (sum_j P|tS|)|O| + |mu| sum_j P|v| + |tO|)."""
+    q, k, v, tq, tk, tv = (x[n][0].double().cpu().numpy() for n in wl.TENSOR_ORDER)
+    s = w.softmax_scale
+    M = orc.mask_matrix(w.mode, w.chunk_tokens, w.n_chunks)
+    bO = np.empty(q.shape)
+    btO = np.empty(q.shape)
+    for h in range(q.shape[1]):
+        S = np.where(M, s * q[:, h] @ k[:, h].T, -np.inf)
+        P = np.exp(S - S.max(axis=1, keepdims=True))
+        P /= P.sum(axis=1, keepdims=True)
+        tS = np.where(M, s * (tq[:, h] @ k[:, h].T + q[:, h] @ tk[:, h].T), 0.0)
+        O = P @ v[:, h]
+        mu = (P * tS).sum(axis=1, keepdims=True)
+        tO = (P * (tS - mu)) @ v[:, h] + P @ tv[:, h]
+        av, atv = np.abs(v[:, h]), np.abs(tv[:, h])
+        bO[:, h] = P @ av + np.abs(O)
+        btO[:, h] = (2 * (P * np.abs(tS)) @ av + P @ atv
+                     + (P * np.abs(tS)).sum(axis=1, keepdims=True) * np.abs(O)
+                     + np.abs(mu) * (P @ av) + np.abs(tO))
+    u = 2.0 ** -9
+    return u * bO, u * btO
+
+
 def test_small_custom_scale_and_distributions(cuda_device):
+    # Outside the configs' distributions (peaked softmax, large tangents) the
+    # bf16 rounding of P and U dominates; hold the kernel to twice the
+    # first-order bound of that rounding (plus fp32 accumulation slack).
     w = wl.Workload("scaled", B=1, H=2, d=128, n_chunks=3, chunk_tokens=100, mode=TF,
                     stds=(1.5, 1.5, 1.0, 2.0, 0.5, 1.0), scale=0.2, seed=77)
-    _dense_check(w, cuda_device)
+    x = wl.make_inputs(w, device=cuda_device)
+    o, to, lse = _run(w, x)
+    xc = {k: v.cpu() for k, v in x.items()}
+    O, tO, LSE = orc.attn_jvp_dense(xc["q"], xc["k"], xc["v"], xc["tq"], xc["tk"], xc["tv"],
+                                    w.mode, w.chunk_tokens, w.n_chunks, w.scale)
+    bO, btO = _rounding_bound(x, w)
+    for name, got, ref, b in (("O", o, O, bO), ("tO", to, tO, btO)):
+        err = np.abs(got.double().cpu().numpy()[0] - ref[0])
+        tol = 2.0 * b + 1e-3 * (1.0 + np.abs(ref[0]))
+        assert (err <= tol).all(), f"{name}: max err/tol {(err / tol).max():.3f}"
+    _close("LSE", lse.double().cpu().numpy(), LSE, TOL["bf16"][1])
 
 
 def _sampled_check(w, device, heads=(0, -1), n_random=256, max_rows=None):

@@ -1,0 +1,76 @@
+"""Multi-rank host logic of the benchmark on CPU (gloo, world size 2).
+
+The path shards into independent (batch, head, query-tile) units, so the only
+cross-rank steps are the barrier and the MAX reduction of timings; every rank
+draws its own replica of the inputs. These tests run those steps on two CPU
+processes.
+"""
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    import datetime
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    from attention_jvp_attn_b200 import inputs as wl
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        t = bench.max_over_ranks(10.0 + 5.0 * rank)          # per-rank "ms"
+        seed = bench.rank_seed(wl.FRAMEWISE_TF, rank)
+        x = wl.make_inputs(wl.TINY_F32, seed=seed)["q"]
+        dist.barrier()
+        q.put((rank, t, seed, float(x.flatten()[0])))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_reduce_max_and_distinct_replicas():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(2))
+    # every rank sees the slowest rank's time
+    assert res[0][1] == 15.0 and res[1][1] == 15.0
+    # the ranks draw different inputs
+    assert res[0][2] != res[1][2] and res[0][3] != res[1][3]
+
+
+def test_job_throughput_is_whole_job_over_slowest_rank():
+    sys.path.insert(0, ROOT)
+    import bench
+    # 2 ranks x 3 steps x 1e12 FLOP in 1.5 s (slowest rank) = 4 TFLOP/s
+    assert bench.job_throughput(2, 10**12, 3, 1500.0) == pytest.approx(4.0)
+    assert bench.max_over_ranks(7.5) == 7.5  # no process group: identity
+
+
+def test_reference_arm_other_ranks_exit_without_work():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--gpus", "2", "--steps", "1", "--warmup", "0"],
+                       capture_output=True, text=True, env=env, timeout=120)
+    assert r.returncode == 0
+    assert r.stdout.strip() == ""

@@ -68,6 +68,9 @@ def load(path: str = None) -> ctypes.CDLL:
                                                 ctypes.POINTER(ctypes.c_int32),
                                                 ctypes.POINTER(ctypes.c_uint8), ctypes.c_int32]
         lib.attn_jvp_schedule_tiles.restype = ctypes.c_int32
+        lib.attn_jvp_fwd_noalloc.argtypes = [ctypes.POINTER(Shape), vp, vp, vp, vp, vp, vp,
+                                             Mask, vp, vp, vp, vp]
+        lib.attn_jvp_fwd_noalloc.restype = ctypes.c_int
         lib.attn_jvp_version.argtypes = []
         lib.attn_jvp_version.restype = ctypes.c_int32
         _lib = lib

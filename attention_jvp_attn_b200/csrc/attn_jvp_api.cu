@@ -220,6 +220,70 @@ int launch_f32(const attn_jvp_shape* s, const void* q, const void* k, const void
 
 int64_t round256(int64_t x) { return (x + 255) & ~int64_t(255); }
 
+// ---- allocation-free variant ---------------------------------------------
+// Scratch of attn_jvp_fwd_noalloc: a file-scope device array (one per device
+// that loads the library). Word 0 is the kernel's status word; the rest is
+// reserved. Host code must not pass `g_noalloc_scratch` itself to a kernel (on
+// the host it is only a stand-in symbol): its device address comes from
+// cudaGetSymbolAddress, looked up once per device below.
+constexpr int kNoAllocScratchWords = ATTN_JVP_NOALLOC_SCRATCH_BYTES / 4;
+constexpr int kNoAllocWordsNeeded = 1;
+static __device__ __align__(256) unsigned int g_noalloc_scratch[kNoAllocScratchWords];
+
+struct NoAllocState {
+  bool ready = false;
+  int sm_count = 0;
+  unsigned int* scratch = nullptr;  // device address of g_noalloc_scratch on this device
+};
+NoAllocState g_noalloc[kMaxDevices];
+
+// Per-device set-up without any allocation: device check, tensor-map encoder,
+// kernel attributes and the scratch array's device address.
+int noalloc_state(NoAllocState** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return ATTN_JVP_ERR_NO_DEVICE;
+  }
+  std::lock_guard<std::mutex> lock(g_mu);
+  NoAllocState& st = g_noalloc[dev];
+  if (!st.ready) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&st.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return ATTN_JVP_ERR_CUDA;
+    }
+    if (major != 10 || minor != 0) return ATTN_JVP_ERR_NO_DEVICE;
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+              cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !fn) {
+        cudaGetLastError();
+        return ATTN_JVP_ERR_CUDA;
+      }
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_noalloc_scratch) != cudaSuccess || addr == nullptr) {
+      cudaGetLastError();
+      return ATTN_JVP_ERR_CUDA;
+    }
+    if (ajvp::tc_prepare(128) != cudaSuccess || ajvp::tc_prepare(64) != cudaSuccess) {
+      cudaGetLastError();
+      return ATTN_JVP_ERR_CUDA;
+    }
+    st.scratch = static_cast<unsigned int*>(addr);
+    st.ready = true;
+  }
+  *out = &st;
+  return ATTN_JVP_OK;
+}
+
+
 }  // namespace
 
 extern "C" {
@@ -345,6 +409,47 @@ int32_t attn_jvp_schedule_tiles(attn_jvp_mask mask, int64_t L, int32_t block_m, 
 }
 
 int32_t attn_jvp_version(void) { return 100; }
+
+int attn_jvp_fwd_noalloc(const attn_jvp_shape* shape, const void* q, const void* k,
+                         const void* v, const void* tq, const void* tk, const void* tv,
+                         attn_jvp_mask mask, void* o, void* to, float* lse, void* stream) {
+  int rc = validate(shape, mask);
+  if (rc != ATTN_JVP_OK) return rc;
+  if (shape->dtype != ATTN_JVP_BF16) return ATTN_JVP_ERR_UNSUPPORTED;
+  if (kNoAllocWordsNeeded > kNoAllocScratchWords) return ATTN_JVP_ERR_UNSUPPORTED;
+  const void* ptrs[9] = {q, k, v, tq, tk, tv, o, to, lse};
+  for (const void* ptr : ptrs)
+    if (!ptr) return ATTN_JVP_ERR_INVALID_ARGUMENT;
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return ATTN_JVP_ERR_MISALIGNED;
+  NoAllocState* st = nullptr;
+  rc = noalloc_state(&st);
+  if (rc != ATTN_JVP_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // The shared word keeps the previous call's value: clear it first.
+  if (cudaMemsetAsync(st->scratch, 0, kNoAllocWordsNeeded * sizeof(unsigned int), s) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_JVP_ERR_CUDA;
+  }
+  DeviceState launch_state;
+  launch_state.ready = true;
+  launch_state.sm_count = st->sm_count;
+  launch_state.status = st->scratch;
+  rc = launch_bf16(&launch_state, shape, q, k, v, tq, tk, tv, mask, o, to, lse, s);
+  if (rc != ATTN_JVP_OK) return rc;
+  if (cudaStreamSynchronize(s) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_JVP_ERR_CUDA;
+  }
+  unsigned int word = 0;
+  if (cudaMemcpy(&word, st->scratch, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_JVP_ERR_CUDA;
+  }
+  return word != 0 ? ATTN_JVP_ERR_DEVICE_TIMEOUT : ATTN_JVP_OK;
+}
+
 
 #ifdef AJVP_TRACE
 // Trace builds only: device buffer of kTraceTiles x kTraceEvents int64 clocks

@@ -155,6 +155,43 @@ int attn_jvp_sync_status(void* stream);
 /* Static, NUL-terminated description of a status code. */
 const char* attn_jvp_status_string(int status);
 
+/*
+ * attn_jvp_fwd_noalloc - attn_jvp_fwd for callers that cannot allocate device
+ * memory (an allocator-free runtime, a plugin host that owns every device
+ * buffer, code running where cudaMalloc is forbidden or would break a memory
+ * budget). It allocates nothing itself: not on the first call, not later.
+ * There is no counterpart in the pages; it is an addition of this library.
+ *
+ * The bf16 kernel needs one word of scratch device memory besides its inputs
+ * and outputs: the status word that a bounded wait sets when it runs out.
+ * attn_jvp_fwd keeps that word in memory the library allocates once per
+ * device. This entry point instead uses a fixed file-scope device array of
+ * ATTN_JVP_NOALLOC_SCRATCH_BYTES bytes (ATTN_JVP_NOALLOC_SCRATCH_BYTES / 4
+ * words, of which this version uses 1), which every GPU that loads the
+ * library holds until the process exits. The scratch does not grow with the
+ * problem; the entry point rejects any layout that would need more words than
+ * the array holds with ATTN_JVP_ERR_UNSUPPORTED, and rejects problems the
+ * kernels cannot run exactly as attn_jvp_fwd does.
+ *
+ * Only bf16 is accepted (the fp32 kernel needs no scratch; use attn_jvp_fwd).
+ * Arguments, layout and outputs are those of attn_jvp_fwd. Unlike it, this
+ * call clears the scratch word on `stream`, launches, waits for `stream` and
+ * returns the status of the launched work, so a bounded-wait timeout is
+ * reported here as ATTN_JVP_ERR_DEVICE_TIMEOUT.
+ *
+ * The first call on a device (with that device current) looks up the array's
+ * device address and the kernels' launch attributes; make that first call
+ * before any stream capture. All calls share the one array: calls that
+ * overlap on the GPU (other threads or streams) race on it.
+ */
+#define ATTN_JVP_NOALLOC_SCRATCH_BYTES 256
+int attn_jvp_fwd_noalloc(const attn_jvp_shape* shape,
+                         const void* q, const void* k, const void* v,
+                         const void* tq, const void* tk, const void* tv,
+                         attn_jvp_mask mask,
+                         void* o, void* to, float* lse,
+                         void* stream);
+
 /* ---- host-side helpers (need no GPU) ---------------------------------- */
 
 /* Number of admissible (query, key) pairs per (batch, head):

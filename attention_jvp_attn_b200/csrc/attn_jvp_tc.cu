@@ -78,7 +78,7 @@ struct TcCfg {
   static constexpr int QBYTES = BM * D * 2;       // bytes of the Q (or tQ) tile
   static constexpr int NSLOT = (D == 128) ? 5 : 10;
   static constexpr int DATA = 2 * QBYTES + NSLOT * TILE;
-  static constexpr int XCH = 2 * BM * 4;          // row-statistics exchange, [2][BM] floats
+  static constexpr int XCH = 2 * BM * 4 + 32;     // row statistics [2][BM] floats + flags [2][4]
   static constexpr int NBAR = 2 * NSLOT + 9 + 8;
   static constexpr int BYTES = 1024 + DATA + XCH + NBAR * 8 + 16;
   static constexpr int HALF = BN / 2;             // key columns per softmax warpgroup
@@ -178,6 +178,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
   uint8_t* sRing = smem + 2 * C::QBYTES;
   float* xch = reinterpret_cast<float*>(smem + C::DATA);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::DATA + C::XCH);
+  volatile uint32_t* xflags = reinterpret_cast<volatile uint32_t*>(xch + 2 * C::BM);
   uint64_t* full = bars;
   uint64_t* empty = bars + C::NSLOT;
   uint64_t* q_full = bars + 2 * C::NSLOT + 0;
@@ -216,6 +217,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
     for (int i = 0; i < 4; ++i) {
       mbar_init(&xa[i], 64);
       mbar_init(&xb[i], 64);
+      xflags[i] = 0;
+      xflags[4 + i] = 0;
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -426,7 +429,44 @@ mma_scores<D, C::BM, C::BN>(tmem + C::TM_TS, aQ, aTK, idesc_s, true);
     const uint32_t tT = tmem + lane_off + C::TM_T + C::DH * wg;
     float* my_x = xch + wg * C::BM + row;
     const float* other_x = xch + (1 - wg) * C::BM + row;
-    uint32_t xa_ph = 0, xb_ph = 0;
+    uint32_t xa_ph = 0, xb_ph = 0, xseq = 0;
+    volatile uint32_t* my_flag = xflags + 4 * wg + sub;
+    volatile uint32_t* other_flag = xflags + 4 * (1 - wg) + sub;
+    // Per-tile swap of the row maxima: one flag round trip. A single buffer is
+    // enough: a warpgroup writes its next tile's value only after that tile's
+    // S is ready, which needs the other warpgroup's P of this tile, which it
+    // arrives on only after reading this value. Bounded spin.
+    auto exchange_max = [&](float mine, float& theirs) -> bool {
+      *my_x = mine;
+      __syncwarp();
+      ++xseq;
+      int ok = 1;
+      if (lane == 0) {
+        __threadfence_block();
+        *my_flag = xseq;
+        uint32_t polls = 0;
+        uint64_t t0 = 0;
+        while (static_cast<int>(*other_flag - xseq) < 0) {
+          if ((++polls & 63u) == 0) {
+            if (*abort_flag) { ok = 0; break; }
+            const uint64_t now = globaltimer_ns();
+            if (t0 == 0) t0 = now;
+            if (now - t0 > kWaitTimeoutNs) {
+              *abort_flag = 1;
+              atomicOr(p.status, kStatusTimeout);
+              ok = 0;
+              break;
+            }
+          }
+        }
+        __threadfence_block();
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      __syncwarp();
+      if (!ok) return false;
+      theirs = *other_x;
+      return true;
+    };
     // Swap one float per row with the other warpgroup (warps sub and sub + 4
     // share rows): write, both arrive, read, both arrive. Bounded waits.
     auto exchange = [&](float mine, float& theirs) -> bool {
@@ -491,7 +531,7 @@ mma_scores<D, C::BM, C::BN>(tmem + C::TM_TS, aQ, aTK, idesc_s, true);
         // row maximum over both halves of the tile
         float their_max;
         tc_fence_before();
-        if (!exchange(my_max, their_max)) { ok = false; break; }
+        if (!exchange_max(my_max, their_max)) { ok = false; break; }
         tc_fence_after();
         const float row_max = fmaxf(my_max, their_max);
         if (warp == 0 && lane == 0) AJVP_EV(g, 6);

@@ -79,7 +79,11 @@ struct TcCfg {
   static constexpr int NSLOT = (D == 128) ? 5 : 10;
   static constexpr int DATA = 2 * QBYTES + NSLOT * TILE;
   static constexpr int XCH = 2 * BM * 4 + 32;     // row statistics [2][BM] floats + flags [2][4]
+#ifdef AJVP_TRACE
+  static constexpr int NBAR = 2 * NSLOT + 9 + 8 + 4;
+#else
   static constexpr int NBAR = 2 * NSLOT + 9 + 8;
+#endif
   static constexpr int BYTES = 1024 + DATA + XCH + NBAR * 8 + 16;
   static constexpr int HALF = BN / 2;             // key columns per softmax warpgroup
   static constexpr int DH = D / 2;                // output columns per softmax warpgroup
@@ -192,6 +196,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
   uint64_t* drain = bars + 2 * C::NSLOT + 8;
   uint64_t* xa = bars + 2 * C::NSLOT + 9;   // [4] row-statistics exchange, first half
   uint64_t* xb = bars + 2 * C::NSLOT + 13;  // [4] second half
+#ifdef AJVP_TRACE
+  uint64_t* obs = bars + 2 * C::NSLOT + 17;  // [4] MMA-group completion, watched by the observer
+#endif
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -219,6 +226,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
       mbar_init(&xb[i], 64);
       xflags[i] = 0;
       xflags[4 + i] = 0;
+#ifdef AJVP_TRACE
+      mbar_init(&obs[i], 1);
+#endif
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -232,6 +242,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+#ifdef AJVP_TRACE
+  if (warp == 8 && lane == 1 && p.trace && blockIdx.x == kTraceCta) {
+    // observer: completion clocks of the MMA groups of each tile
+    for (int g = 0; g < kTraceTiles; ++g) {
+      for (int i = 0; i < 4; ++i) {
+        if (!mbar_wait_drain(&obs[i], g & 1, 2000000000ull)) { g = kTraceTiles; break; }
+        p.trace[g * kTraceEvents + 10 + i] = static_cast<long long>(clock64());
+      }
+    }
+  }
+#endif
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     // Load order per key tile matches the MMA issuer's first use: K, tK, tV, V.
@@ -321,14 +342,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
         if (ok) {
           tc_fence_after();
           const uint32_t aK = slot_addr(0);
-mma_scores<D, C::BM, C::BN>(tmem + C::TM_S, aQ, aK, idesc_s, false);
+          mma_scores<D, C::BM, C::BN>(tmem + C::TM_S, aQ, aK, idesc_s, false);
           umma_commit(s_full);
           ok = mbar_wait(&full[1], 0, abort_flag, p.status);
           if (ok) {
             tc_fence_after();
             const uint32_t aTK = slot_addr(1);
-mma_scores<D, C::BM, C::BN>(tmem + C::TM_TS, aTQ, aK, idesc_s, false);
-mma_scores<D, C::BM, C::BN>(tmem + C::TM_TS, aQ, aTK, idesc_s, true);
+            mma_scores<D, C::BM, C::BN>(tmem + C::TM_TS, aTQ, aK, idesc_s, false);
+            mma_scores<D, C::BM, C::BN>(tmem + C::TM_TS, aQ, aTK, idesc_s, true);
             umma_commit(ts_full);
             umma_commit(&empty[0]);
             umma_commit(&empty[1]);
@@ -361,11 +382,17 @@ mma_scores<D, C::BM, C::BN>(tmem + C::TM_TS, aQ, aTK, idesc_s, true);
           AJVP_EV(g, 1);
           if (!mbar_wait(&full[(c0 + 2) % C::NSLOT], slot_ph(c0 + 2), abort_flag, p.status)) break;
           tc_fence_after();
-mma_values_split<C::BN>(tmem + C::TM_T, tmem + C::TM_S, aTV, idesc_v, idx > 0);
+          mma_values_split<C::BN>(tmem + C::TM_T, tmem + C::TM_S, aTV, idesc_v, idx > 0);
+#ifdef AJVP_TRACE
+          if (p.trace && blockIdx.x == kTraceCta) umma_commit(&obs[0]);
+#endif
           umma_commit(&empty[(c0 + 2) % C::NSLOT]);
           if (!mbar_wait(&full[(c0 + 3) % C::NSLOT], slot_ph(c0 + 3), abort_flag, p.status)) break;
           tc_fence_after();
-mma_values_split<C::BN>(tmem + C::TM_A, tmem + C::TM_S, aV, idesc_v, idx > 0);
+          mma_values_split<C::BN>(tmem + C::TM_A, tmem + C::TM_S, aV, idesc_v, idx > 0);
+#ifdef AJVP_TRACE
+          if (p.trace && blockIdx.x == kTraceCta) umma_commit(&obs[1]);
+#endif
           // S_{g+1}
           if (has_next) {
             if (new_item) {
@@ -375,8 +402,11 @@ mma_values_split<C::BN>(tmem + C::TM_A, tmem + C::TM_S, aV, idesc_v, idx > 0);
             if (!mbar_wait(&full[c1 % C::NSLOT], slot_ph(c1), abort_flag, p.status)) break;
             tc_fence_after();
             const uint32_t aK = slot_addr(c1);
-mma_scores<D, C::BM, C::BN>(tmem + C::TM_S, aQ, aK, idesc_s, false);
+            mma_scores<D, C::BM, C::BN>(tmem + C::TM_S, aQ, aK, idesc_s, false);
             umma_commit(s_full);
+#ifdef AJVP_TRACE
+            if (p.trace && blockIdx.x == kTraceCta) umma_commit(&obs[2]);
+#endif
             AJVP_EV(g, 2);
           }
           // T += U V
@@ -384,7 +414,10 @@ mma_scores<D, C::BM, C::BN>(tmem + C::TM_S, aQ, aK, idesc_s, false);
           u_ph ^= 1;
           AJVP_EV(g, 3);
           tc_fence_after();
-mma_values_split<C::BN>(tmem + C::TM_T, tmem + C::TM_TS, aV, idesc_v, true);
+          mma_values_split<C::BN>(tmem + C::TM_T, tmem + C::TM_TS, aV, idesc_v, true);
+#ifdef AJVP_TRACE
+          if (p.trace && blockIdx.x == kTraceCta) umma_commit(&obs[3]);
+#endif
           umma_commit(&empty[(c0 + 3) % C::NSLOT]);
           umma_commit(uv_done);
           if (idx == cnt - 1) umma_commit(acc_full);
@@ -394,8 +427,8 @@ mma_values_split<C::BN>(tmem + C::TM_T, tmem + C::TM_TS, aV, idesc_v, true);
           tc_fence_after();
           {
             const uint32_t aK = slot_addr(c1), aTK = slot_addr(c1 + 1);
-mma_scores<D, C::BM, C::BN>(tmem + C::TM_TS, aTQ, aK, idesc_s, false);
-mma_scores<D, C::BM, C::BN>(tmem + C::TM_TS, aQ, aTK, idesc_s, true);
+            mma_scores<D, C::BM, C::BN>(tmem + C::TM_TS, aTQ, aK, idesc_s, false);
+            mma_scores<D, C::BM, C::BN>(tmem + C::TM_TS, aQ, aTK, idesc_s, true);
           }
           umma_commit(ts_full);
           AJVP_EV(g, 4);

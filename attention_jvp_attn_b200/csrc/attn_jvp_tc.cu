@@ -10,8 +10,10 @@
 // (128 keys), with s the softmax scale and x = s log2(e) Q K^T:
 //   MMA   S_j   = Q K_j^T                      (TMEM cols [0,128),   fp32)
 //   MMA   tS'_j = tQ K_j^T + Q tK_j^T          (TMEM cols [128,256), fp32)
-//   warps p = 2^(x - m), l += sum p, written back over S as bf16 P
-//         u = p * s * tS', D += sum u,  written back over tS' as bf16 U
+//   warps p = 2^(x - m), l += sum p;  u = p * s * tS', D += sum u;
+//         P and U (bf16) written back over tS' (each warpgroup's 64 columns:
+//         32 of P, then 32 of U), which frees the S columns for S_{j+1}
+//         while the softmax of tile j is still running
 //   MMA   A += P V_j                           (TMEM cols [256,256+d))
 //   MMA   T += U V_j + P tV_j                  (TMEM cols [256+d,256+2d))
 //   end   O = A/l, mu = D/l, tO = T/l - mu O, LSE = (m + log2 l) ln 2
@@ -80,15 +82,17 @@ struct TcCfg {
   static constexpr int DATA = 2 * QBYTES + NSLOT * TILE;
   static constexpr int XCH = 2 * BM * 4 + 32;     // row statistics [2][BM] floats + flags [2][4]
 #ifdef AJVP_TRACE
-  static constexpr int NBAR = 2 * NSLOT + 9 + 8 + 4;
+  static constexpr int NBAR = 2 * NSLOT + 10 + 8 + 4;
 #else
-  static constexpr int NBAR = 2 * NSLOT + 9 + 8;
+  static constexpr int NBAR = 2 * NSLOT + 10 + 8;
 #endif
   static constexpr int BYTES = 1024 + DATA + XCH + NBAR * 8 + 16;
   static constexpr int HALF = BN / 2;             // key columns per softmax warpgroup
   static constexpr int DH = D / 2;                // output columns per softmax warpgroup
   static constexpr uint32_t TM_S = 0;
   static constexpr uint32_t TM_TS = 128;
+  static constexpr uint32_t TM_P = TM_TS;       // bf16 P over the first half of each warpgroup's tS'
+  static constexpr uint32_t TM_U = TM_TS + 32;  // bf16 U over the second half
   static constexpr uint32_t TM_A = 256;
   static constexpr uint32_t TM_T = 256 + D;
   static constexpr uint32_t TM_COLS = 512;
@@ -172,7 +176,7 @@ __device__ __forceinline__ WorkItem decode_item(const TcParams& p, int pos) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid_constant__ TcParams p) {
+__global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_constant__ TcParams p) {
   using C = TcCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -194,10 +198,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
   uint64_t* acc_full = bars + 2 * C::NSLOT + 6;
   uint64_t* uv_done = bars + 2 * C::NSLOT + 7;
   uint64_t* drain = bars + 2 * C::NSLOT + 8;
-  uint64_t* xa = bars + 2 * C::NSLOT + 9;   // [4] row-statistics exchange, first half
-  uint64_t* xb = bars + 2 * C::NSLOT + 13;  // [4] second half
+  uint64_t* s_free = bars + 2 * C::NSLOT + 9;
+  uint64_t* xa = bars + 2 * C::NSLOT + 10;  // [4] row-statistics exchange, first half
+  uint64_t* xb = bars + 2 * C::NSLOT + 14;  // [4] second half
 #ifdef AJVP_TRACE
-  uint64_t* obs = bars + 2 * C::NSLOT + 17;  // [4] MMA-group completion, watched by the observer
+  uint64_t* obs = bars + 2 * C::NSLOT + 18;  // [4] MMA-group completion, watched by the observer ([2] unused)
 #endif
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -221,6 +226,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
     mbar_init(acc_full, 1);
     mbar_init(uv_done, 1);
     mbar_init(drain, 1);
+    mbar_init(s_free, 8);
     for (int i = 0; i < 4; ++i) {
       mbar_init(&xa[i], 64);
       mbar_init(&xb[i], 64);
@@ -244,9 +250,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
 
 #ifdef AJVP_TRACE
   if (warp == 8 && lane == 1 && p.trace && blockIdx.x == kTraceCta) {
-    // observer: completion clocks of the MMA groups of each tile
+    // observer: completion clocks of P tV, P V and U V of each tile (events
+    // 10, 11, 13; S may complete before or after them and is not observed)
     for (int g = 0; g < kTraceTiles; ++g) {
       for (int i = 0; i < 4; ++i) {
+        if (i == 2) continue;
         if (!mbar_wait_drain(&obs[i], g & 1, 2000000000ull)) { g = kTraceTiles; break; }
         p.trace[g * kTraceEvents + 10 + i] = static_cast<long long>(clock64());
       }
@@ -313,20 +321,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
     __syncwarp();
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    // Per key tile g (slots 4g..4g+3 hold K_g, tK_g, tV_g, V_g), in issue order:
-    //   T (+)= P_g tV_g,  A (+)= P_g V_g,  S_{g+1} = Q K_{g+1}^T,
-    //   T += U_g V_g,  tS'_{g+1} = tQ K_{g+1}^T + Q tK_{g+1}^T
-    // so the softmax warps compute U_g while P_g's products and S_{g+1} run,
-    // and P_{g+1} while U_g V_g and tS'_{g+1} run. tcgen05.mma from one thread
-    // execute in order, so S_{g+1} (over P_g's columns) follows every read of
-    // P_g and tS'_{g+1} (over U_g's columns) follows U_g V_g.
+    // Per key tile g (slots 4g..4g+3 hold K_g, tK_g, tV_g, V_g):
+    //   S_{g+1} = Q K_{g+1}^T        once the softmax has read S_g (s_free)
+    //   T (+)= P_g tV_g,  A (+)= P_g V_g          after P_g (p_full)
+    //   T += U_g V_g                               after U_g (u_full)
+    //   tS'_{g+1} = tQ K_{g+1}^T + Q tK_{g+1}^T
+    // S_{g+1} thus runs while the softmax still works on tile g, and the
+    // softmax computes P_{g+1} while P_g's and U_g's products and tS'_{g+1}
+    // run. tcgen05.mma from one thread execute in order, so tS'_{g+1} (over
+    // the columns of P_g and U_g) follows every read of them.
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(C::BM, C::BN, 0);
       const uint32_t idesc_v = idesc_bf16_f32(C::BM, D, 1);
       const uint32_t aQ = smem_u32(sQ), aTQ = smem_u32(sTQ), aRing = smem_u32(sRing);
       auto slot_addr = [&](uint32_t c) { return aRing + (c % C::NSLOT) * C::TILE; };
       auto slot_ph = [&](uint32_t c) { return (c / C::NSLOT) & 1; };
-      uint32_t q_ph = 0, p_ph = 0, u_ph = 0;
+      uint32_t q_ph = 0, p_ph = 0, u_ph = 0, sf_ph = 0;
       bool ok = true;
       int k = 0, pos = 0;
       if (next_item(p, cta, G, k, pos)) {
@@ -375,46 +385,53 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
           }
           const uint32_t c0 = 4 * g, c1 = 4 * (g + 1);
           const uint32_t aTV = slot_addr(c0 + 2), aV = slot_addr(c0 + 3);
-          // T (+)= P tV, A (+)= P V
-          AJVP_EV(g, 0);
+          // S_{g+1} goes out as soon as the softmax warps have taken S_g out of
+          // TMEM and K_{g+1} has landed: polled (never waited for) between the
+          // groups of this tile, waited for before tS'_{g+1} if still pending.
+          // A new item's first S waits for its Q there too.
+          bool s_done = !has_next;
+#define AJVP_ISSUE_S()                                                                     \
+  do {                                                                                     \
+    tc_fence_after();                                                                      \
+    mma_scores<D, C::BM, C::BN>(tmem + C::TM_S, aQ, slot_addr(c1), idesc_s, false);        \
+    umma_commit(s_full);                                                                   \
+    AJVP_EV(g, 0);                                                                         \
+    s_done = true;                                                                         \
+  } while (0)
+#define AJVP_POLL_S()                                                                      \
+  do {                                                                                     \
+    if (!s_done && !new_item && mbar_test_wait(s_free, sf_ph) &&                           \
+        mbar_test_wait(&full[c1 % C::NSLOT], slot_ph(c1))) {                               \
+      sf_ph ^= 1;                                                                          \
+      AJVP_ISSUE_S();                                                                      \
+    }                                                                                      \
+  } while (0)
+          AJVP_POLL_S();
+          // T (+)= P_g tV_g, A (+)= P_g V_g
+          if (!mbar_wait(&full[(c0 + 2) % C::NSLOT], slot_ph(c0 + 2), abort_flag, p.status)) break;
+          if (!mbar_wait(&full[(c0 + 3) % C::NSLOT], slot_ph(c0 + 3), abort_flag, p.status)) break;
+          AJVP_POLL_S();
           if (!mbar_wait(p_full, p_ph, abort_flag, p.status)) break;
           p_ph ^= 1;
           AJVP_EV(g, 1);
-          if (!mbar_wait(&full[(c0 + 2) % C::NSLOT], slot_ph(c0 + 2), abort_flag, p.status)) break;
           tc_fence_after();
-          mma_values_split<C::BN>(tmem + C::TM_T, tmem + C::TM_S, aTV, idesc_v, idx > 0);
+          mma_values_split<C::BN>(tmem + C::TM_T, tmem + C::TM_P, aTV, idesc_v, idx > 0);
 #ifdef AJVP_TRACE
           if (p.trace && blockIdx.x == kTraceCta) umma_commit(&obs[0]);
 #endif
           umma_commit(&empty[(c0 + 2) % C::NSLOT]);
-          if (!mbar_wait(&full[(c0 + 3) % C::NSLOT], slot_ph(c0 + 3), abort_flag, p.status)) break;
-          tc_fence_after();
-          mma_values_split<C::BN>(tmem + C::TM_A, tmem + C::TM_S, aV, idesc_v, idx > 0);
+          mma_values_split<C::BN>(tmem + C::TM_A, tmem + C::TM_P, aV, idesc_v, idx > 0);
 #ifdef AJVP_TRACE
           if (p.trace && blockIdx.x == kTraceCta) umma_commit(&obs[1]);
 #endif
-          // S_{g+1}
-          if (has_next) {
-            if (new_item) {
-              if (!mbar_wait(q_full, q_ph, abort_flag, p.status)) break;
-              q_ph ^= 1;
-            }
-            if (!mbar_wait(&full[c1 % C::NSLOT], slot_ph(c1), abort_flag, p.status)) break;
-            tc_fence_after();
-            const uint32_t aK = slot_addr(c1);
-            mma_scores<D, C::BM, C::BN>(tmem + C::TM_S, aQ, aK, idesc_s, false);
-            umma_commit(s_full);
-#ifdef AJVP_TRACE
-            if (p.trace && blockIdx.x == kTraceCta) umma_commit(&obs[2]);
-#endif
-            AJVP_EV(g, 2);
-          }
-          // T += U V
+          AJVP_EV(g, 2);
+          AJVP_POLL_S();
+          // T += U_g V_g
           if (!mbar_wait(u_full, u_ph, abort_flag, p.status)) break;
           u_ph ^= 1;
           AJVP_EV(g, 3);
           tc_fence_after();
-          mma_values_split<C::BN>(tmem + C::TM_T, tmem + C::TM_TS, aV, idesc_v, true);
+          mma_values_split<C::BN>(tmem + C::TM_T, tmem + C::TM_U, aV, idesc_v, true);
 #ifdef AJVP_TRACE
           if (p.trace && blockIdx.x == kTraceCta) umma_commit(&obs[3]);
 #endif
@@ -422,7 +439,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
           umma_commit(uv_done);
           if (idx == cnt - 1) umma_commit(acc_full);
           if (!has_next) break;
-          // tS'_{g+1}
+          if (!s_done) {
+            if (new_item) {
+              if (!mbar_wait(q_full, q_ph, abort_flag, p.status)) break;
+              q_ph ^= 1;
+            }
+            if (!mbar_wait(s_free, sf_ph, abort_flag, p.status)) break;
+            sf_ph ^= 1;
+            if (!mbar_wait(&full[c1 % C::NSLOT], slot_ph(c1), abort_flag, p.status)) break;
+            AJVP_ISSUE_S();
+          }
+          // tS'_{g+1}, over the columns of P_g and U_g (read by the MMAs above)
           if (!mbar_wait(&full[(c1 + 1) % C::NSLOT], slot_ph(c1 + 1), abort_flag, p.status)) break;
           tc_fence_after();
           {
@@ -435,6 +462,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
           umma_commit(&empty[c1 % C::NSLOT]);
           umma_commit(&empty[(c1 + 1) % C::NSLOT]);
           if (idx2 == cnt2 - 1) umma_commit(q_empty);
+#undef AJVP_POLL_S
+#undef AJVP_ISSUE_S
           w = w2;
           sch = sch2;
           cnt = cnt2;
@@ -467,8 +496,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
     volatile uint32_t* other_flag = xflags + 4 * (1 - wg) + sub;
     // Per-tile swap of the row maxima: one flag round trip. A single buffer is
     // enough: a warpgroup writes its next tile's value only after that tile's
-    // S is ready, which needs the other warpgroup's P of this tile, which it
-    // arrives on only after reading this value. Bounded spin.
+    // S is ready, and that S is issued only once every softmax warp has
+    // arrived on s_free, which each does after reading this value. Bounded spin.
     auto exchange_max = [&](float mine, float& theirs) -> bool {
       *my_x = mine;
       __syncwarp();
@@ -565,6 +594,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
         float their_max;
         tc_fence_before();
         if (!exchange_max(my_max, their_max)) { ok = false; break; }
+        // S_g is in registers and both warpgroups have read this tile's maxima:
+        // the MMA warp may write S_{g+1} over S_g.
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free);
         tc_fence_after();
         const float row_max = fmaxf(my_max, their_max);
         if (warp == 0 && lane == 0) AJVP_EV(g, 6);
@@ -581,8 +614,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
           resc = true;
         }
         if (__any_sync(0xffffffffu, resc)) {
-          // A: every P V of earlier tiles is complete (S of this tile was
-          // issued after it). T: wait for the U V of the previous tile.
+          // Every value MMA of earlier tiles has completed once the previous
+          // tile's U V has (they run in issue order).
+          if (!warp_wait(uv_done, (g - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
 #pragma unroll 1
           for (int c = 0; c < C::DH / 32; ++c) {
             uint32_t a[32];
@@ -592,8 +627,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
             for (int j = 0; j < 32; ++j) a[j] = __float_as_uint(__uint_as_float(a[j]) * alpha);
             tmem_st32(tA + 32 * c, a);
           }
-          if (!warp_wait(uv_done, (g - 1) & 1, abort_flag, p.status)) { ok = false; break; }
-          tc_fence_after();
 #pragma unroll 1
           for (int c = 0; c < C::DH / 32; ++c) {
             uint32_t a[32];
@@ -621,42 +654,47 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_jvp_tc_kernel(const __grid
           pk[j + 1] = pack_bf16x2(p2, p3);
         }
         l += (ls0 + ls1) + (ls2 + ls3);
-        tmem_st32(tS, pk);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(p_full);
         if (warp == 0 && lane == 0) AJVP_EV(g, 7);
 
         if (!warp_wait(ts_full, ts_ph, abort_flag, p.status)) { ok = false; break; }
         ts_ph ^= 1;
         if (warp == 0 && lane == 0) AJVP_EV(g, 8);
         tc_fence_after();
-        uint32_t v[C::HALF];
-        tmem_ld32(tTS, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-        tmem_ld32(tTS + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        // tS' in two halves of 32 keys: P goes over the first half once it
+        // is read, U over the second.
+        uint32_t v[32];
+        tmem_ld32(tTS, v);
         tmem_wait_ld();
+        tmem_st32(tTS, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full);
         uint32_t uk[C::HALF / 2];
         float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
+        // u = p s tS' for keys [32 h, 32 h + 32) of this warpgroup's half tile
+        auto u_half = [&](int h) {
 #pragma unroll
-        for (int j = 0; j < C::HALF / 2; j += 2) {
-          const float q0 = bf16lo_to_f32(pk[j]) * scale;
-          const float q1 = bf16hi_to_f32(pk[j]) * scale;
-          const float q2 = bf16lo_to_f32(pk[j + 1]) * scale;
-          const float q3 = bf16hi_to_f32(pk[j + 1]) * scale;
-          const float u0 = q0 * __uint_as_float(v[2 * j]);
-          const float u1 = q1 * __uint_as_float(v[2 * j + 1]);
-          const float u2 = q2 * __uint_as_float(v[2 * j + 2]);
-          const float u3 = q3 * __uint_as_float(v[2 * j + 3]);
-          d0 += u0;
-          d1 += u1;
-          d2 += u2;
-          d3 += u3;
-          uk[j] = pack_bf16x2(u0, u1);
-          uk[j + 1] = pack_bf16x2(u2, u3);
-        }
+          for (int j = 0; j < 16; j += 2) {
+            const uint32_t pa = pk[16 * h + j], pb = pk[16 * h + j + 1];
+            const float u0 = bf16lo_to_f32(pa) * scale * __uint_as_float(v[2 * j]);
+            const float u1 = bf16hi_to_f32(pa) * scale * __uint_as_float(v[2 * j + 1]);
+            const float u2 = bf16lo_to_f32(pb) * scale * __uint_as_float(v[2 * j + 2]);
+            const float u3 = bf16hi_to_f32(pb) * scale * __uint_as_float(v[2 * j + 3]);
+            d0 += u0;
+            d1 += u1;
+            d2 += u2;
+            d3 += u3;
+            uk[16 * h + j] = pack_bf16x2(u0, u1);
+            uk[16 * h + j + 1] = pack_bf16x2(u2, u3);
+          }
+        };
+        u_half(0);
+        tmem_ld32(tTS + 32, v);
+        tmem_wait_ld();
+        u_half(1);
         dsum += (d0 + d1) + (d2 + d3);
-        tmem_st32(tTS, uk);
+        tmem_st32(tTS + 32, uk);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();

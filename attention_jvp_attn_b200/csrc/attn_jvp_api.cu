@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstddef>
 #include <cstring>
@@ -25,6 +26,7 @@ struct DeviceState {
   bool ready = false;
   int status_code = ATTN_JVP_OK;  // why the device is unusable, if it is
   int sm_count = 0;
+  int pair_clusters = 0;           // CTA pairs resident at once (0: pair kernel unavailable)
   unsigned int* status = nullptr;  // device status word (bit 0: a bounded wait ran out)
 };
 
@@ -36,6 +38,7 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn g_encode = nullptr;
+std::atomic<int> g_use_pairs{0};  // d = 128 runs on CTA pairs when switched on
 #ifdef AJVP_TRACE
 long long* g_trace = nullptr;
 #endif
@@ -84,6 +87,7 @@ int device_state(DeviceState** out) {
       st.status = nullptr;
       return ATTN_JVP_ERR_CUDA;
     }
+    st.pair_clusters = ajvp::tc_pair_max_clusters(st.sm_count);
     st.ready = true;
   }
   *out = &st;
@@ -146,12 +150,12 @@ MaskSpec mask_spec(attn_jvp_mask m, int64_t L) {
   return ms;
 }
 
-// Query tiles of one head, most key tiles first (stable among equals).
-int fill_order(const MaskSpec& ms, int n_qtiles, uint16_t* order) {
+// Query row blocks (of `bm` rows) of one head, most key tiles first (stable among equals).
+int fill_order(const MaskSpec& ms, int n_qtiles, int bm, uint16_t* order) {
   if (n_qtiles > ajvp::kMaxOrder) return 0;
   std::vector<int> cost(n_qtiles), idx(n_qtiles);
   for (int t = 0; t < n_qtiles; ++t) {
-    cost[t] = ajvp::make_tile_sched(ms, t, ajvp::kTcBlockM, ajvp::kTcBlockN).count();
+    cost[t] = ajvp::make_tile_sched(ms, t, bm, ajvp::kTcBlockN).count();
     idx[t] = t;
   }
   std::stable_sort(idx.begin(), idx.end(), [&](int a, int b) { return cost[a] > cost[b]; });
@@ -164,11 +168,15 @@ int launch_bf16(DeviceState* st, const attn_jvp_shape* s, const void* q, const v
                 void* o, void* to, float* lse, cudaStream_t stream) {
   static thread_local ajvp::TcParams p;  // large (order table): not on the stack
   std::memset(&p, 0, offsetof(ajvp::TcParams, order));
+  // CTA pairs (d = 128): each CTA loads 64 of the 128 keys of a K or tK tile.
+  const bool pair = s->d == 128 && st->pair_clusters > 0 && g_use_pairs.load() != 0;
+  const int k_rows = pair ? ajvp::kTcBlockN / 2 : ajvp::kTcBlockN;
+  const int bmu = pair ? 2 * ajvp::kTcBlockM : ajvp::kTcBlockM;
   if (!encode_bf16_map(&p.map_q, q, s, ajvp::kTcBlockM) ||
-      !encode_bf16_map(&p.map_k, k, s, ajvp::kTcBlockN) ||
+      !encode_bf16_map(&p.map_k, k, s, k_rows) ||
       !encode_bf16_map(&p.map_v, v, s, ajvp::kTcBlockN) ||
       !encode_bf16_map(&p.map_tq, tq, s, ajvp::kTcBlockM) ||
-      !encode_bf16_map(&p.map_tk, tk, s, ajvp::kTcBlockN) ||
+      !encode_bf16_map(&p.map_tk, tk, s, k_rows) ||
       !encode_bf16_map(&p.map_tv, tv, s, ajvp::kTcBlockN))
     return ATTN_JVP_ERR_CUDA;
   p.o = o;
@@ -178,18 +186,19 @@ int launch_bf16(DeviceState* st, const attn_jvp_shape* s, const void* q, const v
   p.B = static_cast<int>(s->B);
   p.H = static_cast<int>(s->H);
   p.L = static_cast<int>(s->L);
-  p.n_qtiles = static_cast<int>((s->L + ajvp::kTcBlockM - 1) / ajvp::kTcBlockM);
+  p.n_qtiles = static_cast<int>((s->L + bmu - 1) / bmu);
   p.n_items = p.B * p.H * p.n_qtiles;
   p.mask = mask_spec(mask, s->L);
   const float sc = softmax_scale(s);
   p.scale = sc;
   p.scale_log2 = sc * 1.4426950408889634f;
-  p.order_len = fill_order(p.mask, p.n_qtiles, p.order);
+  p.order_len = fill_order(p.mask, p.n_qtiles, bmu, p.order);
 #ifdef AJVP_TRACE
   p.trace = g_trace;
 #endif
-  const int grid = std::min(st->sm_count, p.n_items);
-  if (ajvp::tc_launch(static_cast<int>(s->d), p, grid, stream) != cudaSuccess)
+  const int grid = pair ? 2 * std::min(st->pair_clusters, p.n_items)
+                        : std::min(st->sm_count, p.n_items);
+  if (ajvp::tc_launch(static_cast<int>(s->d), pair, p, grid, stream) != cudaSuccess)
     return ATTN_JVP_ERR_CUDA;
   return ATTN_JVP_OK;
 }
@@ -233,6 +242,7 @@ static __device__ __align__(256) unsigned int g_noalloc_scratch[kNoAllocScratchW
 struct NoAllocState {
   bool ready = false;
   int sm_count = 0;
+  int pair_clusters = 0;
   unsigned int* scratch = nullptr;  // device address of g_noalloc_scratch on this device
 };
 NoAllocState g_noalloc[kMaxDevices];
@@ -277,6 +287,7 @@ int noalloc_state(NoAllocState** out) {
       return ATTN_JVP_ERR_CUDA;
     }
     st.scratch = static_cast<unsigned int*>(addr);
+    st.pair_clusters = ajvp::tc_pair_max_clusters(st.sm_count);
     st.ready = true;
   }
   *out = &st;
@@ -435,6 +446,7 @@ int attn_jvp_fwd_noalloc(const attn_jvp_shape* shape, const void* q, const void*
   DeviceState launch_state;
   launch_state.ready = true;
   launch_state.sm_count = st->sm_count;
+  launch_state.pair_clusters = st->pair_clusters;
   launch_state.status = st->scratch;
   rc = launch_bf16(&launch_state, shape, q, k, v, tq, tk, tv, mask, o, to, lse, s);
   if (rc != ATTN_JVP_OK) return rc;
@@ -450,6 +462,8 @@ int attn_jvp_fwd_noalloc(const attn_jvp_shape* shape, const void* q, const void*
   return word != 0 ? ATTN_JVP_ERR_DEVICE_TIMEOUT : ATTN_JVP_OK;
 }
 
+
+int attn_jvp_set_cta_pairs(int enable) { return g_use_pairs.exchange(enable ? 1 : 0); }
 
 #ifdef AJVP_TRACE
 // Trace builds only: device buffer of kTraceTiles x kTraceEvents int64 clocks

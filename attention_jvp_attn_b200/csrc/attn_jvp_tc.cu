@@ -71,14 +71,23 @@ __device__ __forceinline__ long long clock_after(float x) {
   } while (0)
 #endif
 
-template <int D>
+// PAIR: a cluster of two CTAs runs cta_group::2 MMAs over 256 query rows
+// (128 per CTA); each CTA holds half of every K/V-type tile: 64 of the 128
+// keys of K and tK, 64 of the D columns of V and tV.
+template <int D, bool PAIR>
 struct TcCfg {
-  static constexpr int BM = kTcBlockM;
+  static constexpr int BM = kTcBlockM;            // query rows per CTA
+  static constexpr int BMU = PAIR ? 2 * BM : BM;  // query rows per work item
   static constexpr int BN = kTcBlockN;
   static constexpr int CH = D / 64;               // 128-byte swizzle chunks per row
-  static constexpr int TILE = BN * D * 2;         // bytes of one K/V-type tile
+  static constexpr int KROWS = PAIR ? BN / 2 : BN;  // key rows of a K-type tile held here
+  static constexpr int VCH = PAIR ? CH / 2 : CH;    // 64-column chunks of a V-type tile held here
+  static constexpr int TILE = KROWS * D * 2;      // bytes of one K/V-type tile (or half tile)
   static constexpr int QBYTES = BM * D * 2;       // bytes of the Q (or tQ) tile
-  static constexpr int NSLOT = (D == 128) ? 5 : 10;
+  static constexpr int NSLOT = (TILE == 32768) ? 5 : 10;
+  static constexpr int M_MMA = PAIR ? 2 * BM : BM;
+  static_assert(!PAIR || D == 128, "CTA pairs split d = 128 into two 64-column chunks");
+  static_assert(KROWS * D == BN * VCH * 64, "K-type and V-type tiles fill a slot alike");
   static constexpr int DATA = 2 * QBYTES + NSLOT * TILE;
   static constexpr int XCH = 2 * BM * 4 + 32;     // row statistics [2][BM] floats + flags [2][4]
 #ifdef AJVP_TRACE
@@ -87,6 +96,7 @@ struct TcCfg {
   static constexpr int NBAR = 2 * NSLOT + 10 + 8;
 #endif
   static constexpr int BYTES = 1024 + DATA + XCH + NBAR * 8 + 16;
+  static constexpr int ARRIVALS = PAIR ? 16 : 8;  // softmax warps arriving on s_free, p_full, u_full
   static constexpr int HALF = BN / 2;             // key columns per softmax warpgroup
   static constexpr int DH = D / 2;                // output columns per softmax warpgroup
   static constexpr uint32_t TM_S = 0;
@@ -118,7 +128,7 @@ __device__ __forceinline__ uint32_t tmem_a_operand(uint32_t base, int ks) {
 // Score MMA: D[tmem] (+)= A B^T over the head dimension, A a [rows_a x D]
 // and B a [rows_b x D] K-major tile. Offsets are added to the descriptors'
 // start-address field (16-byte units; tiles lie well inside its 256 KB range).
-template <int D, int ROWS_A, int ROWS_B>
+template <int D, int ROWS_A, int ROWS_B, bool PAIR>
 __device__ __forceinline__ void mma_scores(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem,
                                            uint32_t idesc, bool accumulate) {
   const uint64_t da = smem_desc_sw128(a_smem, 16, 1024);
@@ -127,20 +137,28 @@ __device__ __forceinline__ void mma_scores(uint32_t d_tmem, uint32_t a_smem, uin
   for (int kk = 0; kk < D / 16; ++kk) {
     const uint32_t oa = ((kk >> 2) * ROWS_A * 128 + (kk & 3) * 32) >> 4;
     const uint32_t ob = ((kk >> 2) * ROWS_B * 128 + (kk & 3) * 32) >> 4;
-    umma_ss(d_tmem, da + oa, db + ob, idesc, (accumulate || kk > 0) ? 1u : 0u);
+    if constexpr (PAIR)
+      umma_ss_pair(d_tmem, da + oa, db + ob, idesc, (accumulate || kk > 0) ? 1u : 0u);
+    else
+      umma_ss(d_tmem, da + oa, db + ob, idesc, (accumulate || kk > 0) ? 1u : 0u);
   }
 }
 
 // Value MMA: D[tmem] (+)= P[tmem] V, P a bf16 [128 x BN] tile in TMEM (in the
-// two-warpgroup layout of tmem_a_operand) and V a [BN keys x D] tile read MN-major.
-template <int BN>
+// two-warpgroup layout of tmem_a_operand) and V a [BN keys x D] tile read
+// MN-major (for a pair, each CTA holds one 64-column chunk of it).
+template <int BN, bool PAIR>
 __device__ __forceinline__ void mma_values_split(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem,
                                            uint32_t idesc, bool accumulate) {
   const uint64_t db = smem_desc_sw128(b_smem, BN * 128, 1024);
 #pragma unroll
-  for (int ks = 0; ks < BN / 16; ++ks)
-    umma_ts(d_tmem, tmem_a_operand(a_tmem, ks), db + ((ks * 16 * 128) >> 4), idesc,
-            (accumulate || ks > 0) ? 1u : 0u);
+  for (int ks = 0; ks < BN / 16; ++ks) {
+    const uint32_t acc = (accumulate || ks > 0) ? 1u : 0u;
+    if constexpr (PAIR)
+      umma_ts_pair(d_tmem, tmem_a_operand(a_tmem, ks), db + ((ks * 16 * 128) >> 4), idesc, acc);
+    else
+      umma_ts(d_tmem, tmem_a_operand(a_tmem, ks), db + ((ks * 16 * 128) >> 4), idesc, acc);
+  }
 }
 
 // Bit mask of the lowest n bits (n clamped to [0, 32]).
@@ -175,9 +193,9 @@ __device__ __forceinline__ WorkItem decode_item(const TcParams& p, int pos) {
   return w;
 }
 
-template <int D>
+template <int D, bool PAIR>
 __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_constant__ TcParams p) {
-  using C = TcCfg<D>;
+  using C = TcCfg<D, PAIR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -209,8 +227,29 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int G = gridDim.x;
-  const int cta = blockIdx.x;
+  // Work is distributed over units: single CTAs, or CTA pairs (clusters of 2).
+  const int G = PAIR ? gridDim.x / 2 : gridDim.x;
+  const int cta = PAIR ? blockIdx.x / 2 : blockIdx.x;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;  // 0: issues the MMAs
+  const bool mma_cta = rank == 0;
+  // Barriers the leader waits on and other threads (of either CTA) arrive on.
+  auto leader_addr = [&](uint64_t* bar) -> uint32_t {
+    return PAIR ? mapa_shared(smem_u32(bar), 0) : smem_u32(bar);
+  };
+  auto arrive_leader = [&](uint64_t* bar) {
+    if constexpr (PAIR)
+      mbar_arrive_cluster(leader_addr(bar));
+    else
+      mbar_arrive(bar);
+  };
+  auto bwait = [&](uint64_t* bar, uint32_t parity) -> bool {
+    return PAIR ? mbar_wait_cluster(bar, parity, abort_flag, p.status)
+                : mbar_wait(bar, parity, abort_flag, p.status);
+  };
+  auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
+    return PAIR ? warp_wait_cluster(bar, parity, abort_flag, p.status)
+                : warp_wait(bar, parity, abort_flag, p.status);
+  };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NSLOT; ++i) {
@@ -221,12 +260,12 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
     mbar_init(q_empty, 1);
     mbar_init(s_full, 1);
     mbar_init(ts_full, 1);
-    mbar_init(p_full, 8);
-    mbar_init(u_full, 8);
+    mbar_init(p_full, C::ARRIVALS);
+    mbar_init(u_full, C::ARRIVALS);
     mbar_init(acc_full, 1);
     mbar_init(uv_done, 1);
     mbar_init(drain, 1);
-    mbar_init(s_free, 8);
+    mbar_init(s_free, C::ARRIVALS);
     for (int i = 0; i < 4; ++i) {
       mbar_init(&xa[i], 64);
       mbar_init(&xb[i], 64);
@@ -240,16 +279,24 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
     fence_barrier_init();
   }
   if (warp == 9) {
-    tmem_alloc(tmem_slot, C::TM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, C::TM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, C::TM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR)
+    cluster_sync_all();  // both CTAs' barriers exist before any remote arrive
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
 #ifdef AJVP_TRACE
-  if (warp == 8 && lane == 1 && p.trace && blockIdx.x == kTraceCta) {
+  if (!PAIR && warp == 8 && lane == 1 && p.trace && blockIdx.x == kTraceCta) {
     // observer: completion clocks of P tV, P V and U V of each tile (events
     // 10, 11, 13; S may complete before or after them and is not observed)
     for (int g = 0; g < kTraceTiles; ++g) {
@@ -264,6 +311,8 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     // Load order per key tile matches the MMA issuer's first use: K, tK, tV, V.
+    // In a pair both CTAs load their halves; the copies complete on the
+    // leader's barriers, which only the leader's producer arms (for both).
     if (lane == 0) {
       tma_prefetch_desc(&p.map_q);
       tma_prefetch_desc(&p.map_k);
@@ -272,7 +321,9 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
       tma_prefetch_desc(&p.map_tk);
       tma_prefetch_desc(&p.map_tv);
       const uint64_t keep = l2_policy_evict_last();
+      [[maybe_unused]] const uint64_t once = l2_policy_evict_first();
       const CUtensorMap* kv_maps[4] = {&p.map_k, &p.map_tk, &p.map_tv, &p.map_v};
+      const uint32_t arm = PAIR ? 2u : 1u;  // CTAs whose copies complete on one barrier
       uint32_t ctr = 0, q_issued = 0, q_ph = 0;
       bool ok = true;
       int k = 0, pos = 0;
@@ -280,17 +331,25 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
         ++k;
         const WorkItem w = decode_item(p, pos);
         if (q_issued > 0) {
-          if (!mbar_wait(q_empty, q_ph, abort_flag, p.status)) { ok = false; break; }
+          if (!bwait(q_empty, q_ph)) { ok = false; break; }
           q_ph ^= 1;
         }
-        mbar_arrive_expect_tx(q_full, 2 * C::QBYTES);
+        if (mma_cta) mbar_arrive_expect_tx(q_full, arm * 2 * C::QBYTES);
+        const int q_row = w.qt * C::BMU + static_cast<int>(rank) * C::BM;
 #pragma unroll
         for (int c = 0; c < C::CH; ++c) {
-          tma_load_4d(sQ + c * C::BM * 128, &p.map_q, q_full, c * 64, w.h, w.qt * C::BM, w.b);
-          tma_load_4d(sTQ + c * C::BM * 128, &p.map_tq, q_full, c * 64, w.h, w.qt * C::BM, w.b);
+          if constexpr (PAIR) {
+            tma_load_4d_pair(sQ + c * C::BM * 128, &p.map_q, leader_addr(q_full), c * 64, w.h, q_row,
+                             w.b, once);
+            tma_load_4d_pair(sTQ + c * C::BM * 128, &p.map_tq, leader_addr(q_full), c * 64, w.h,
+                             q_row, w.b, once);
+          } else {
+            tma_load_4d(sQ + c * C::BM * 128, &p.map_q, q_full, c * 64, w.h, q_row, w.b);
+            tma_load_4d(sTQ + c * C::BM * 128, &p.map_tq, q_full, c * 64, w.h, q_row, w.b);
+          }
         }
         ++q_issued;
-        const TileSched sch = make_tile_sched(p.mask, w.qt, C::BM, C::BN);
+        const TileSched sch = make_tile_sched(p.mask, w.qt, C::BMU, C::BN);
         const int cnt = sch.count();
         for (int idx = 0; ok && idx < cnt; ++idx) {
           const int kt = sch.tile(idx);
@@ -298,24 +357,46 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
           for (int u = 0; u < 4; ++u) {
             const uint32_t slot = ctr % C::NSLOT;
             const uint32_t ph = (ctr / C::NSLOT) & 1;
-            if (!mbar_wait(&empty[slot], ph ^ 1, abort_flag, p.status)) { ok = false; break; }
-            mbar_arrive_expect_tx(&full[slot], C::TILE);
+            if (!bwait(&empty[slot], ph ^ 1)) { ok = false; break; }
+            if (mma_cta) mbar_arrive_expect_tx(&full[slot], arm * C::TILE);
             uint8_t* dst = sRing + slot * C::TILE;
+            if constexpr (PAIR) {
+              if (u < 2) {
+                // K, tK: keys [64 rank, 64 rank + 64) of the tile, all D columns
 #pragma unroll
-            for (int c = 0; c < C::CH; ++c)
-              tma_load_4d_hint(dst + c * C::BN * 128, kv_maps[u], &full[slot], c * 64, w.h,
-                               kt * C::BN, w.b, keep);
+                for (int c = 0; c < C::CH; ++c)
+                  tma_load_4d_pair(dst + c * C::KROWS * 128, kv_maps[u], leader_addr(&full[slot]),
+                                   c * 64, w.h, kt * C::BN + static_cast<int>(rank) * C::KROWS, w.b,
+                                   keep);
+              } else {
+                // V, tV: all keys of the tile, columns [64 rank, 64 rank + 64)
+                tma_load_4d_pair(dst, kv_maps[u], leader_addr(&full[slot]),
+                                 static_cast<int>(rank) * 64, w.h, kt * C::BN, w.b, keep);
+              }
+            } else {
+#pragma unroll
+              for (int c = 0; c < C::CH; ++c)
+                tma_load_4d_hint(dst + c * C::BN * 128, kv_maps[u], &full[slot], c * 64, w.h,
+                                 kt * C::BN, w.b, keep);
+            }
             ++ctr;
           }
         }
       }
       if (!ok) {
-        // Abort: let every copy already issued land before the CTA exits.
-        for (uint32_t s = 0; s < C::NSLOT && s < ctr; ++s) {
-          const uint32_t last = ctr - 1 - ((ctr - 1 + C::NSLOT - s) % C::NSLOT);
-          mbar_wait_drain(&full[s], (last / C::NSLOT) & 1, 200000000ull);
+        if constexpr (PAIR) {
+          // Abort: the copies complete on the leader's barriers, so wait for
+          // them by time (they depend on nothing but memory) before exiting.
+          const uint64_t t0 = globaltimer_ns();
+          while (globaltimer_ns() - t0 < 2000000ull) __nanosleep(1000);
+        } else {
+          // Abort: let every copy already issued land before the CTA exits.
+          for (uint32_t s = 0; s < C::NSLOT && s < ctr; ++s) {
+            const uint32_t last = ctr - 1 - ((ctr - 1 + C::NSLOT - s) % C::NSLOT);
+            mbar_wait_drain(&full[s], (last / C::NSLOT) & 1, 200000000ull);
+          }
+          if (q_issued > 0) mbar_wait_drain(q_full, (q_issued - 1) & 1, 200000000ull);
         }
-        if (q_issued > 0) mbar_wait_drain(q_full, (q_issued - 1) & 1, 200000000ull);
       }
     }
     __syncwarp();
@@ -330,9 +411,21 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
     // softmax computes P_{g+1} while P_g's and U_g's products and tS'_{g+1}
     // run. tcgen05.mma from one thread execute in order, so tS'_{g+1} (over
     // the columns of P_g and U_g) follows every read of them.
-    if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16_f32(C::BM, C::BN, 0);
-      const uint32_t idesc_v = idesc_bf16_f32(C::BM, D, 1);
+    // In a pair only the leader's warp 9 issues; its commits arrive on the
+    // barriers of both CTAs.
+    auto commit_all = [&](uint64_t* bar) {
+      if constexpr (PAIR) {
+        umma_commit_pair_both(bar);
+      } else {
+        umma_commit(bar);
+      }
+    };
+    auto poll = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return PAIR ? mbar_test_wait_cluster(bar, parity) : mbar_test_wait(bar, parity);
+    };
+    if (lane == 0 && mma_cta) {
+      const uint32_t idesc_s = idesc_bf16_f32(C::M_MMA, C::BN, 0);
+      const uint32_t idesc_v = idesc_bf16_f32(C::M_MMA, D, 1);
       const uint32_t aQ = smem_u32(sQ), aTQ = smem_u32(sTQ), aRing = smem_u32(sRing);
       auto slot_addr = [&](uint32_t c) { return aRing + (c % C::NSLOT) * C::TILE; };
       auto slot_ph = [&](uint32_t c) { return (c / C::NSLOT) & 1; };
@@ -342,28 +435,28 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
       if (next_item(p, cta, G, k, pos)) {
         ++k;
         WorkItem w = decode_item(p, pos);
-        TileSched sch = make_tile_sched(p.mask, w.qt, C::BM, C::BN);
+        TileSched sch = make_tile_sched(p.mask, w.qt, C::BMU, C::BN);
         int cnt = sch.count(), idx = 0;
         uint32_t g = 0;
         // prologue: scores of the first tile
-        ok = mbar_wait(q_full, q_ph, abort_flag, p.status);
+        ok = bwait(q_full, q_ph);
         q_ph ^= 1;
-        if (ok) ok = mbar_wait(&full[0], 0, abort_flag, p.status);
+        if (ok) ok = bwait(&full[0], 0);
         if (ok) {
           tc_fence_after();
           const uint32_t aK = slot_addr(0);
-          mma_scores<D, C::BM, C::BN>(tmem + C::TM_S, aQ, aK, idesc_s, false);
-          umma_commit(s_full);
-          ok = mbar_wait(&full[1], 0, abort_flag, p.status);
+          mma_scores<D, C::BM, C::KROWS, PAIR>(tmem + C::TM_S, aQ, aK, idesc_s, false);
+          commit_all(s_full);
+          ok = bwait(&full[1], 0);
           if (ok) {
             tc_fence_after();
             const uint32_t aTK = slot_addr(1);
-            mma_scores<D, C::BM, C::BN>(tmem + C::TM_TS, aTQ, aK, idesc_s, false);
-            mma_scores<D, C::BM, C::BN>(tmem + C::TM_TS, aQ, aTK, idesc_s, true);
-            umma_commit(ts_full);
-            umma_commit(&empty[0]);
-            umma_commit(&empty[1]);
-            if (cnt == 1) umma_commit(q_empty);
+            mma_scores<D, C::BM, C::KROWS, PAIR>(tmem + C::TM_TS, aTQ, aK, idesc_s, false);
+            mma_scores<D, C::BM, C::KROWS, PAIR>(tmem + C::TM_TS, aQ, aTK, idesc_s, true);
+            commit_all(ts_full);
+            commit_all(&empty[0]);
+            commit_all(&empty[1]);
+            if (cnt == 1) commit_all(q_empty);
           }
         }
         while (ok) {
@@ -377,7 +470,7 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
             if (has_next) {
               ++k;
               w2 = decode_item(p, pos);
-              sch2 = make_tile_sched(p.mask, w2.qt, C::BM, C::BN);
+              sch2 = make_tile_sched(p.mask, w2.qt, C::BMU, C::BN);
               cnt2 = sch2.count();
               idx2 = 0;
               new_item = true;
@@ -393,75 +486,75 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
 #define AJVP_ISSUE_S()                                                                     \
   do {                                                                                     \
     tc_fence_after();                                                                      \
-    mma_scores<D, C::BM, C::BN>(tmem + C::TM_S, aQ, slot_addr(c1), idesc_s, false);        \
-    umma_commit(s_full);                                                                   \
+    mma_scores<D, C::BM, C::KROWS, PAIR>(tmem + C::TM_S, aQ, slot_addr(c1), idesc_s, false);        \
+    commit_all(s_full);                                                                   \
     AJVP_EV(g, 0);                                                                         \
     s_done = true;                                                                         \
   } while (0)
 #define AJVP_POLL_S()                                                                      \
   do {                                                                                     \
-    if (!s_done && !new_item && mbar_test_wait(s_free, sf_ph) &&                           \
-        mbar_test_wait(&full[c1 % C::NSLOT], slot_ph(c1))) {                               \
+    if (!s_done && !new_item && poll(s_free, sf_ph) &&                           \
+        poll(&full[c1 % C::NSLOT], slot_ph(c1))) {                               \
       sf_ph ^= 1;                                                                          \
       AJVP_ISSUE_S();                                                                      \
     }                                                                                      \
   } while (0)
           AJVP_POLL_S();
           // T (+)= P_g tV_g, A (+)= P_g V_g
-          if (!mbar_wait(&full[(c0 + 2) % C::NSLOT], slot_ph(c0 + 2), abort_flag, p.status)) break;
-          if (!mbar_wait(&full[(c0 + 3) % C::NSLOT], slot_ph(c0 + 3), abort_flag, p.status)) break;
+          if (!bwait(&full[(c0 + 2) % C::NSLOT], slot_ph(c0 + 2))) break;
+          if (!bwait(&full[(c0 + 3) % C::NSLOT], slot_ph(c0 + 3))) break;
           AJVP_POLL_S();
-          if (!mbar_wait(p_full, p_ph, abort_flag, p.status)) break;
+          if (!bwait(p_full, p_ph)) break;
           p_ph ^= 1;
           AJVP_EV(g, 1);
           tc_fence_after();
-          mma_values_split<C::BN>(tmem + C::TM_T, tmem + C::TM_P, aTV, idesc_v, idx > 0);
+          mma_values_split<C::BN, PAIR>(tmem + C::TM_T, tmem + C::TM_P, aTV, idesc_v, idx > 0);
 #ifdef AJVP_TRACE
-          if (p.trace && blockIdx.x == kTraceCta) umma_commit(&obs[0]);
+          if (!PAIR && p.trace && blockIdx.x == kTraceCta) commit_all(&obs[0]);
 #endif
-          umma_commit(&empty[(c0 + 2) % C::NSLOT]);
-          mma_values_split<C::BN>(tmem + C::TM_A, tmem + C::TM_P, aV, idesc_v, idx > 0);
+          commit_all(&empty[(c0 + 2) % C::NSLOT]);
+          mma_values_split<C::BN, PAIR>(tmem + C::TM_A, tmem + C::TM_P, aV, idesc_v, idx > 0);
 #ifdef AJVP_TRACE
-          if (p.trace && blockIdx.x == kTraceCta) umma_commit(&obs[1]);
+          if (!PAIR && p.trace && blockIdx.x == kTraceCta) commit_all(&obs[1]);
 #endif
           AJVP_EV(g, 2);
           AJVP_POLL_S();
           // T += U_g V_g
-          if (!mbar_wait(u_full, u_ph, abort_flag, p.status)) break;
+          if (!bwait(u_full, u_ph)) break;
           u_ph ^= 1;
           AJVP_EV(g, 3);
           tc_fence_after();
-          mma_values_split<C::BN>(tmem + C::TM_T, tmem + C::TM_U, aV, idesc_v, true);
+          mma_values_split<C::BN, PAIR>(tmem + C::TM_T, tmem + C::TM_U, aV, idesc_v, true);
 #ifdef AJVP_TRACE
-          if (p.trace && blockIdx.x == kTraceCta) umma_commit(&obs[3]);
+          if (!PAIR && p.trace && blockIdx.x == kTraceCta) commit_all(&obs[3]);
 #endif
-          umma_commit(&empty[(c0 + 3) % C::NSLOT]);
-          umma_commit(uv_done);
-          if (idx == cnt - 1) umma_commit(acc_full);
+          commit_all(&empty[(c0 + 3) % C::NSLOT]);
+          commit_all(uv_done);
+          if (idx == cnt - 1) commit_all(acc_full);
           if (!has_next) break;
           if (!s_done) {
             if (new_item) {
-              if (!mbar_wait(q_full, q_ph, abort_flag, p.status)) break;
+              if (!bwait(q_full, q_ph)) break;
               q_ph ^= 1;
             }
-            if (!mbar_wait(s_free, sf_ph, abort_flag, p.status)) break;
+            if (!bwait(s_free, sf_ph)) break;
             sf_ph ^= 1;
-            if (!mbar_wait(&full[c1 % C::NSLOT], slot_ph(c1), abort_flag, p.status)) break;
+            if (!bwait(&full[c1 % C::NSLOT], slot_ph(c1))) break;
             AJVP_ISSUE_S();
           }
           // tS'_{g+1}, over the columns of P_g and U_g (read by the MMAs above)
-          if (!mbar_wait(&full[(c1 + 1) % C::NSLOT], slot_ph(c1 + 1), abort_flag, p.status)) break;
+          if (!bwait(&full[(c1 + 1) % C::NSLOT], slot_ph(c1 + 1))) break;
           tc_fence_after();
           {
             const uint32_t aK = slot_addr(c1), aTK = slot_addr(c1 + 1);
-            mma_scores<D, C::BM, C::BN>(tmem + C::TM_TS, aTQ, aK, idesc_s, false);
-            mma_scores<D, C::BM, C::BN>(tmem + C::TM_TS, aQ, aTK, idesc_s, true);
+            mma_scores<D, C::BM, C::KROWS, PAIR>(tmem + C::TM_TS, aTQ, aK, idesc_s, false);
+            mma_scores<D, C::BM, C::KROWS, PAIR>(tmem + C::TM_TS, aQ, aTK, idesc_s, true);
           }
-          umma_commit(ts_full);
+          commit_all(ts_full);
           AJVP_EV(g, 4);
-          umma_commit(&empty[c1 % C::NSLOT]);
-          umma_commit(&empty[(c1 + 1) % C::NSLOT]);
-          if (idx2 == cnt2 - 1) umma_commit(q_empty);
+          commit_all(&empty[c1 % C::NSLOT]);
+          commit_all(&empty[(c1 + 1) % C::NSLOT]);
+          if (idx2 == cnt2 - 1) commit_all(q_empty);
 #undef AJVP_POLL_S
 #undef AJVP_ISSUE_S
           w = w2;
@@ -472,7 +565,10 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
         }
       }
       // Every MMA issued so far completes before TMEM is released.
-      umma_commit(drain);
+      if constexpr (PAIR)
+        umma_commit_pair(drain);
+      else
+        umma_commit(drain);
       mbar_wait_drain(drain, 0, 1000000000ull);
     }
     __syncwarp();
@@ -550,16 +646,16 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
     while (ok && next_item(p, cta, G, k, pos)) {
       ++k;
       const WorkItem w = decode_item(p, pos);
-      const int t = w.qt * C::BM + row;  // this thread's query row
+      const int t = w.qt * C::BMU + static_cast<int>(rank) * C::BM + row;  // this thread's query row
       const RowRange rr = row_range(p.mask, t);
-      const TileSched sch = make_tile_sched(p.mask, w.qt, C::BM, C::BN);
+      const TileSched sch = make_tile_sched(p.mask, w.qt, C::BMU, C::BN);
       const int cnt = sch.count();
       float m_use = -INFINITY, l = 0.f, dsum = 0.f;
       for (int idx = 0; idx < cnt; ++idx, ++g) {
         const int kt = sch.tile(idx);
         const bool full_tile = sch.full(kt);
         const int k0 = kt * C::BN + C::HALF * wg;
-        if (!warp_wait(s_full, s_ph, abort_flag, p.status)) { ok = false; break; }
+        if (!wwait(s_full, s_ph)) { ok = false; break; }
         s_ph ^= 1;
         if (warp == 0 && lane == 0) AJVP_EV(g, 5);
         tc_fence_after();
@@ -597,7 +693,7 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
         // S_g is in registers and both warpgroups have read this tile's maxima:
         // the MMA warp may write S_{g+1} over S_g.
         __syncwarp();
-        if (lane == 0) mbar_arrive(s_free);
+        if (lane == 0) arrive_leader(s_free);
         tc_fence_after();
         const float row_max = fmaxf(my_max, their_max);
         if (warp == 0 && lane == 0) AJVP_EV(g, 6);
@@ -616,7 +712,7 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
         if (__any_sync(0xffffffffu, resc)) {
           // Every value MMA of earlier tiles has completed once the previous
           // tile's U V has (they run in issue order).
-          if (!warp_wait(uv_done, (g - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+          if (!wwait(uv_done, (g - 1) & 1)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll 1
           for (int c = 0; c < C::DH / 32; ++c) {
@@ -656,7 +752,7 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
         l += (ls0 + ls1) + (ls2 + ls3);
         if (warp == 0 && lane == 0) AJVP_EV(g, 7);
 
-        if (!warp_wait(ts_full, ts_ph, abort_flag, p.status)) { ok = false; break; }
+        if (!wwait(ts_full, ts_ph)) { ok = false; break; }
         ts_ph ^= 1;
         if (warp == 0 && lane == 0) AJVP_EV(g, 8);
         tc_fence_after();
@@ -669,7 +765,7 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full);
+        if (lane == 0) arrive_leader(p_full);
         uint32_t uk[C::HALF / 2];
         float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
         // u = p s tS' for keys [32 h, 32 h + 32) of this warpgroup's half tile
@@ -698,12 +794,12 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(u_full);
+        if (lane == 0) arrive_leader(u_full);
         if (warp == 0 && lane == 0) AJVP_EV(g, 9);
       }
       if (!ok) break;
       // ---------------- epilogue: O = A/l, tO = T/l - (D/l) O, LSE
-      if (!warp_wait(acc_full, acc_ph, abort_flag, p.status)) { ok = false; break; }
+      if (!wwait(acc_full, acc_ph)) { ok = false; break; }
       acc_ph ^= 1;
       tc_fence_after();
       float l_other, d_other;
@@ -751,26 +847,77 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
     tc_fence_before();
   }
 
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 9) tmem_dealloc(tmem, C::TM_COLS);
+  if constexpr (PAIR) {
+    // Neither CTA leaves (or frees its TMEM) while the leader's MMAs may still
+    // read the other's shared or tensor memory.
+    cluster_sync_all();
+    tc_fence_after();
+    if (warp == 9) tmem_dealloc_pair(tmem, C::TM_COLS);
+  } else {
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 9) tmem_dealloc(tmem, C::TM_COLS);
+  }
 }
 
-size_t tc_smem_bytes(int d) { return d == 128 ? TcCfg<128>::BYTES : TcCfg<64>::BYTES; }
+size_t tc_smem_bytes(int d, bool pair) {
+  if (d == 128) return pair ? TcCfg<128, true>::BYTES : TcCfg<128, false>::BYTES;
+  return TcCfg<64, false>::BYTES;
+}
 
 cudaError_t tc_prepare(int d) {
-  if (d == 128)
-    return cudaFuncSetAttribute(attn_jvp_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                TcCfg<128>::BYTES);
-  return cudaFuncSetAttribute(attn_jvp_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              TcCfg<64>::BYTES);
+  if (d == 128) {
+    cudaError_t e = cudaFuncSetAttribute(attn_jvp_tc_kernel<128, false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         TcCfg<128, false>::BYTES);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(attn_jvp_tc_kernel<128, true>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                TcCfg<128, true>::BYTES);
+  }
+  return cudaFuncSetAttribute(attn_jvp_tc_kernel<64, false>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<64, false>::BYTES);
 }
 
-cudaError_t tc_launch(int d, const TcParams& p, int grid, cudaStream_t stream) {
+namespace {
+void pair_config(cudaLaunchConfig_t* cfg, cudaLaunchAttribute* attr, int grid, cudaStream_t stream) {
+  *cfg = cudaLaunchConfig_t{};
+  cfg->gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg->blockDim = dim3(kTcThreads, 1, 1);
+  cfg->dynamicSmemBytes = TcCfg<128, true>::BYTES;
+  cfg->stream = stream;
+  attr->id = cudaLaunchAttributeClusterDimension;
+  attr->val.clusterDim.x = 2;
+  attr->val.clusterDim.y = 1;
+  attr->val.clusterDim.z = 1;
+  cfg->attrs = attr;
+  cfg->numAttrs = 1;
+}
+}  // namespace
+
+int tc_pair_max_clusters(int sm_count) {
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr;
+  pair_config(&cfg, &attr, 2 * (sm_count / 2), nullptr);
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, attn_jvp_tc_kernel<128, true>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+cudaError_t tc_launch(int d, bool pair, const TcParams& p, int grid, cudaStream_t stream) {
+  if (d == 128 && pair) {
+    cudaLaunchConfig_t cfg;
+    cudaLaunchAttribute attr;
+    pair_config(&cfg, &attr, grid, stream);
+    return cudaLaunchKernelEx(&cfg, attn_jvp_tc_kernel<128, true>, p);
+  }
   if (d == 128)
-    attn_jvp_tc_kernel<128><<<grid, kTcThreads, TcCfg<128>::BYTES, stream>>>(p);
+    attn_jvp_tc_kernel<128, false><<<grid, kTcThreads, TcCfg<128, false>::BYTES, stream>>>(p);
   else
-    attn_jvp_tc_kernel<64><<<grid, kTcThreads, TcCfg<64>::BYTES, stream>>>(p);
+    attn_jvp_tc_kernel<64, false><<<grid, kTcThreads, TcCfg<64, false>::BYTES, stream>>>(p);
   return cudaGetLastError();
 }
 

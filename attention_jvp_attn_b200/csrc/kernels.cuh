@@ -22,7 +22,7 @@ struct TcParams {
   float* lse;
   unsigned int* status;
   int B, H, L;
-  int n_qtiles;  // ceil(L / 128)
+  int n_qtiles;  // query row blocks per (batch, head): ceil(L / 128), or ceil(L / 256) for pairs
   int n_items;   // B * H * n_qtiles
   MaskSpec mask;
   float scale_log2;  // s * log2(e)
@@ -37,12 +37,15 @@ struct TcParams {
 #ifdef AJVP_TRACE
 constexpr int kTraceTiles = 512;
 constexpr int kTraceEvents = 16;
-constexpr int kTraceCta = 5;  // a CTA whose first items are mostly full tiles
+constexpr int kTraceCta = 4;  // a CTA (the leader of a pair) whose first items are mostly full tiles
 #endif
 
-size_t tc_smem_bytes(int d);
-cudaError_t tc_prepare(int d);  // sets the dynamic shared-memory limit (once per device)
-cudaError_t tc_launch(int d, const TcParams& p, int grid, cudaStream_t stream);
+size_t tc_smem_bytes(int d, bool pair);
+cudaError_t tc_prepare(int d);  // sets the dynamic shared-memory limits (once per device)
+// Clusters of two CTAs (the pair kernel, d = 128) that fit on the device at once; 0 if unknown.
+int tc_pair_max_clusters(int sm_count);
+// pair: launch the CTA-pair kernel (d = 128 only) with `grid` CTAs, an even number.
+cudaError_t tc_launch(int d, bool pair, const TcParams& p, int grid, cudaStream_t stream);
 
 // ---- fp32 CUDA-core kernel ----
 constexpr int kSimtBlockQ = 32;

@@ -423,12 +423,22 @@ __device__ __forceinline__ void umma_ts_pair(uint32_t d_tmem, uint32_t a_tmem, u
       : "memory");
 }
 
-// Arrive on the barrier at shared::cluster address `bar_cluster` (either CTA
-// of the pair) once every pair MMA this thread issued so far is done.
-__device__ __forceinline__ void umma_commit_pair(uint32_t bar_cluster) {
+// Arrive on this CTA's barrier `bar` once every pair MMA this thread issued
+// so far is done.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   bar_cluster)
+                   smem_u32(bar))
                : "memory");
+}
+
+// The same completion signalled on the barrier at `bar`'s offset in both CTAs
+// of the pair (a commit, not a copy: no data moves between the CTAs).
+__device__ __forceinline__ void umma_commit_pair_both(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_u32(bar)),
+      "h"(static_cast<uint16_t>(0x3))
+      : "memory");
 }
 
 // ---------------------------------------------------------------- math

@@ -21,7 +21,6 @@ from ._abi import AttnJvpError  # noqa: F401
 from .inputs import BLOCK_CAUSAL, TEACHER_FORCING  # noqa: F401
 
 __all__ = ["attn_jvp", "attn_jvp_host", "sync_status", "unmasked_pairs", "schedule_tiles",
-           "set_cta_pairs",
            "host_staging_bytes", "AttnJvpError", "TEACHER_FORCING", "BLOCK_CAUSAL"]
 
 _DT = {torch.bfloat16: _abi.DTYPE_BF16, torch.float32: _abi.DTYPE_F32}
@@ -109,12 +108,6 @@ def sync_status(device: Optional[torch.device] = None) -> int:
     dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
     with torch.cuda.device(dev):
         return int(_abi.load().attn_jvp_sync_status(_stream_handle(dev)))
-
-
-def set_cta_pairs(enable: bool) -> bool:
-    """Run head-dim-128 bf16 calls on CTA pairs (True) or on single CTAs (False,
-    the default); returns the previous setting. Both give the same result."""
-    return bool(_abi.load().attn_jvp_set_cta_pairs(1 if enable else 0))
 
 
 def unmasked_pairs(mode: int, chunk_tokens: int, n_chunks: int) -> int:

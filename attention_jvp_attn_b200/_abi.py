@@ -71,8 +71,6 @@ def load(path: str = None) -> ctypes.CDLL:
         lib.attn_jvp_fwd_noalloc.argtypes = [ctypes.POINTER(Shape), vp, vp, vp, vp, vp, vp,
                                              Mask, vp, vp, vp, vp]
         lib.attn_jvp_fwd_noalloc.restype = ctypes.c_int
-        lib.attn_jvp_set_cta_pairs.argtypes = [ctypes.c_int]
-        lib.attn_jvp_set_cta_pairs.restype = ctypes.c_int
         lib.attn_jvp_version.argtypes = []
         lib.attn_jvp_version.restype = ctypes.c_int32
         _lib = lib

@@ -4,7 +4,6 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
-#include <atomic>
 #include <cmath>
 #include <cstddef>
 #include <cstring>
@@ -38,7 +37,6 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn g_encode = nullptr;
-std::atomic<int> g_use_pairs{0};  // d = 128 runs on CTA pairs when switched on
 #ifdef AJVP_TRACE
 long long* g_trace = nullptr;
 #endif
@@ -168,8 +166,9 @@ int launch_bf16(DeviceState* st, const attn_jvp_shape* s, const void* q, const v
                 void* o, void* to, float* lse, cudaStream_t stream) {
   static thread_local ajvp::TcParams p;  // large (order table): not on the stack
   std::memset(&p, 0, offsetof(ajvp::TcParams, order));
-  // CTA pairs (d = 128): each CTA loads 64 of the 128 keys of a K or tK tile.
-  const bool pair = s->d == 128 && st->pair_clusters > 0 && g_use_pairs.load() != 0;
+  // d = 128 runs on CTA pairs: each CTA loads 64 of the 128 keys of a K or tK tile.
+  const bool pair = s->d == 128;
+  if (pair && st->pair_clusters <= 0) return ATTN_JVP_ERR_CUDA;
   const int k_rows = pair ? ajvp::kTcBlockN / 2 : ajvp::kTcBlockN;
   const int bmu = pair ? 2 * ajvp::kTcBlockM : ajvp::kTcBlockM;
   if (!encode_bf16_map(&p.map_q, q, s, ajvp::kTcBlockM) ||
@@ -198,7 +197,7 @@ int launch_bf16(DeviceState* st, const attn_jvp_shape* s, const void* q, const v
 #endif
   const int grid = pair ? 2 * std::min(st->pair_clusters, p.n_items)
                         : std::min(st->sm_count, p.n_items);
-  if (ajvp::tc_launch(static_cast<int>(s->d), pair, p, grid, stream) != cudaSuccess)
+  if (ajvp::tc_launch(static_cast<int>(s->d), p, grid, stream) != cudaSuccess)
     return ATTN_JVP_ERR_CUDA;
   return ATTN_JVP_OK;
 }
@@ -462,8 +461,6 @@ int attn_jvp_fwd_noalloc(const attn_jvp_shape* shape, const void* q, const void*
   return word != 0 ? ATTN_JVP_ERR_DEVICE_TIMEOUT : ATTN_JVP_OK;
 }
 
-
-int attn_jvp_set_cta_pairs(int enable) { return g_use_pairs.exchange(enable ? 1 : 0); }
 
 #ifdef AJVP_TRACE
 // Trace builds only: device buffer of kTraceTiles x kTraceEvents int64 clocks

@@ -73,7 +73,10 @@ __device__ __forceinline__ long long clock_after(float x) {
 
 // PAIR: a cluster of two CTAs runs cta_group::2 MMAs over 256 query rows
 // (128 per CTA); each CTA holds half of every K/V-type tile: 64 of the 128
-// keys of K and tK, 64 of the D columns of V and tV.
+// keys of K and tK, 64 of the D columns of V and tV. d = 128 runs on pairs,
+// d = 64 on single CTAs; either way a tile (or half tile) is 16 KB, and the
+// shared-memory ring holds NP elements of two tiles each: (K_j, tK_j) or
+// (tV_j, V_j), each with one full and one empty barrier.
 template <int D, bool PAIR>
 struct TcCfg {
   static constexpr int BM = kTcBlockM;            // query rows per CTA
@@ -84,16 +87,17 @@ struct TcCfg {
   static constexpr int VCH = PAIR ? CH / 2 : CH;    // 64-column chunks of a V-type tile held here
   static constexpr int TILE = KROWS * D * 2;      // bytes of one K/V-type tile (or half tile)
   static constexpr int QBYTES = BM * D * 2;       // bytes of the Q (or tQ) tile
-  static constexpr int NSLOT = (TILE == 32768) ? 5 : 10;
+  static constexpr int NP = 5;                    // ring elements (two tiles each)
   static constexpr int M_MMA = PAIR ? 2 * BM : BM;
-  static_assert(!PAIR || D == 128, "CTA pairs split d = 128 into two 64-column chunks");
+  static_assert(PAIR == (D == 128), "d = 128 runs on CTA pairs, d = 64 on single CTAs");
   static_assert(KROWS * D == BN * VCH * 64, "K-type and V-type tiles fill a slot alike");
-  static constexpr int DATA = 2 * QBYTES + NSLOT * TILE;
+  static_assert(TILE == 16384, "16 KB tiles");
+  static constexpr int DATA = 2 * QBYTES + NP * 2 * TILE;
   static constexpr int XCH = 2 * BM * 4 + 32;     // row statistics [2][BM] floats + flags [2][4]
 #ifdef AJVP_TRACE
-  static constexpr int NBAR = 2 * NSLOT + 10 + 8 + 4;
+  static constexpr int NBAR = 2 * NP + 9 + 8 + 4;
 #else
-  static constexpr int NBAR = 2 * NSLOT + 10 + 8;
+  static constexpr int NBAR = 2 * NP + 9 + 8;
 #endif
   static constexpr int BYTES = 1024 + DATA + XCH + NBAR * 8 + 16;
   static constexpr int ARRIVALS = PAIR ? 16 : 8;  // softmax warps arriving on s_free, p_full, u_full
@@ -128,9 +132,16 @@ __device__ __forceinline__ uint32_t tmem_a_operand(uint32_t base, int ks) {
 // Score MMA: D[tmem] (+)= A B^T over the head dimension, A a [rows_a x D]
 // and B a [rows_b x D] K-major tile. Offsets are added to the descriptors'
 // start-address field (16-byte units; tiles lie well inside its 256 KB range).
-template <int D, int ROWS_A, int ROWS_B, bool PAIR>
+struct NoHook {
+  __device__ __forceinline__ void operator()() const {}
+};
+
+// The MMA helpers call `hook` right after issuing instruction AT (if AT >= 0):
+// the MMA warp tests its next barriers there, so the test's latency overlaps
+// the instructions still to be issued instead of leaving the pipe idle.
+template <int D, int ROWS_A, int ROWS_B, bool PAIR, int AT = -1, typename Hook = NoHook>
 __device__ __forceinline__ void mma_scores(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem,
-                                           uint32_t idesc, bool accumulate) {
+                                           uint32_t idesc, bool accumulate, Hook hook = Hook{}) {
   const uint64_t da = smem_desc_sw128(a_smem, 16, 1024);
   const uint64_t db = smem_desc_sw128(b_smem, 16, 1024);
 #pragma unroll
@@ -141,15 +152,16 @@ __device__ __forceinline__ void mma_scores(uint32_t d_tmem, uint32_t a_smem, uin
       umma_ss_pair(d_tmem, da + oa, db + ob, idesc, (accumulate || kk > 0) ? 1u : 0u);
     else
       umma_ss(d_tmem, da + oa, db + ob, idesc, (accumulate || kk > 0) ? 1u : 0u);
+    if (kk == AT) hook();
   }
 }
 
 // Value MMA: D[tmem] (+)= P[tmem] V, P a bf16 [128 x BN] tile in TMEM (in the
 // two-warpgroup layout of tmem_a_operand) and V a [BN keys x D] tile read
 // MN-major (for a pair, each CTA holds one 64-column chunk of it).
-template <int BN, bool PAIR>
+template <int BN, bool PAIR, int AT = -1, typename Hook = NoHook>
 __device__ __forceinline__ void mma_values_split(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem,
-                                           uint32_t idesc, bool accumulate) {
+                                           uint32_t idesc, bool accumulate, Hook hook = Hook{}) {
   const uint64_t db = smem_desc_sw128(b_smem, BN * 128, 1024);
 #pragma unroll
   for (int ks = 0; ks < BN / 16; ++ks) {
@@ -158,6 +170,7 @@ __device__ __forceinline__ void mma_values_split(uint32_t d_tmem, uint32_t a_tme
       umma_ts_pair(d_tmem, tmem_a_operand(a_tmem, ks), db + ((ks * 16 * 128) >> 4), idesc, acc);
     else
       umma_ts(d_tmem, tmem_a_operand(a_tmem, ks), db + ((ks * 16 * 128) >> 4), idesc, acc);
+    if (ks == AT) hook();
   }
 }
 
@@ -205,22 +218,21 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
   float* xch = reinterpret_cast<float*>(smem + C::DATA);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::DATA + C::XCH);
   volatile uint32_t* xflags = reinterpret_cast<volatile uint32_t*>(xch + 2 * C::BM);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + C::NSLOT;
-  uint64_t* q_full = bars + 2 * C::NSLOT + 0;
-  uint64_t* q_empty = bars + 2 * C::NSLOT + 1;
-  uint64_t* s_full = bars + 2 * C::NSLOT + 2;
-  uint64_t* ts_full = bars + 2 * C::NSLOT + 3;
-  uint64_t* p_full = bars + 2 * C::NSLOT + 4;
-  uint64_t* u_full = bars + 2 * C::NSLOT + 5;
-  uint64_t* acc_full = bars + 2 * C::NSLOT + 6;
-  uint64_t* uv_done = bars + 2 * C::NSLOT + 7;
-  uint64_t* drain = bars + 2 * C::NSLOT + 8;
-  uint64_t* s_free = bars + 2 * C::NSLOT + 9;
-  uint64_t* xa = bars + 2 * C::NSLOT + 10;  // [4] row-statistics exchange, first half
-  uint64_t* xb = bars + 2 * C::NSLOT + 14;  // [4] second half
+  uint64_t* full = bars;            // [NP] ring element landed
+  uint64_t* empty = bars + C::NP;   // [NP] ring element consumed
+  uint64_t* q_full = bars + 2 * C::NP + 0;
+  uint64_t* q_empty = bars + 2 * C::NP + 1;
+  uint64_t* s_full = bars + 2 * C::NP + 2;
+  uint64_t* ts_full = bars + 2 * C::NP + 3;
+  uint64_t* p_full = bars + 2 * C::NP + 4;
+  uint64_t* u_full = bars + 2 * C::NP + 5;
+  uint64_t* acc_full = bars + 2 * C::NP + 6;
+  uint64_t* drain = bars + 2 * C::NP + 7;
+  uint64_t* s_free = bars + 2 * C::NP + 8;
+  uint64_t* xa = bars + 2 * C::NP + 9;   // [4] row-statistics exchange, first half
+  uint64_t* xb = bars + 2 * C::NP + 13;  // [4] second half
 #ifdef AJVP_TRACE
-  uint64_t* obs = bars + 2 * C::NSLOT + 18;  // [4] MMA-group completion, watched by the observer ([2] unused)
+  uint64_t* obs = bars + 2 * C::NP + 17;  // [4] MMA-group completion, watched by the observer ([2] unused)
 #endif
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -237,22 +249,20 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
     return PAIR ? mapa_shared(smem_u32(bar), 0) : smem_u32(bar);
   };
   auto arrive_leader = [&](uint64_t* bar) {
-    if constexpr (PAIR)
-      mbar_arrive_cluster(leader_addr(bar));
+    if (PAIR && rank != 0)
+      mbar_arrive_remote(leader_addr(bar));
     else
       mbar_arrive(bar);
   };
   auto bwait = [&](uint64_t* bar, uint32_t parity) -> bool {
-    return PAIR ? mbar_wait_cluster(bar, parity, abort_flag, p.status)
-                : mbar_wait(bar, parity, abort_flag, p.status);
+    return mbar_wait(bar, parity, abort_flag, p.status);
   };
   auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
-    return PAIR ? warp_wait_cluster(bar, parity, abort_flag, p.status)
-                : warp_wait(bar, parity, abort_flag, p.status);
+    return warp_wait(bar, parity, abort_flag, p.status);
   };
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::NSLOT; ++i) {
+    for (int i = 0; i < C::NP; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
@@ -263,7 +273,6 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
     mbar_init(p_full, C::ARRIVALS);
     mbar_init(u_full, C::ARRIVALS);
     mbar_init(acc_full, 1);
-    mbar_init(uv_done, 1);
     mbar_init(drain, 1);
     mbar_init(s_free, C::ARRIVALS);
     for (int i = 0; i < 4; ++i) {
@@ -310,9 +319,9 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
 #endif
   if (warp == 8) {
     // ------------------------------------------------------------ producer
-    // Load order per key tile matches the MMA issuer's first use: K, tK, tV, V.
-    // In a pair both CTAs load their halves; the copies complete on the
-    // leader's barriers, which only the leader's producer arms (for both).
+    // Ring elements in order of first use: per key tile j, (K_j, tK_j) then
+    // (tV_j, V_j). In a pair both CTAs load their halves; the copies complete
+    // on the leader's barriers, which only the leader's producer arms (for both).
     if (lane == 0) {
       tma_prefetch_desc(&p.map_q);
       tma_prefetch_desc(&p.map_k);
@@ -322,8 +331,29 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
       tma_prefetch_desc(&p.map_tv);
       const uint64_t keep = l2_policy_evict_last();
       [[maybe_unused]] const uint64_t once = l2_policy_evict_first();
-      const CUtensorMap* kv_maps[4] = {&p.map_k, &p.map_tk, &p.map_tv, &p.map_v};
+      const CUtensorMap* maps[2][2] = {{&p.map_k, &p.map_tk}, {&p.map_tv, &p.map_v}};
       const uint32_t arm = PAIR ? 2u : 1u;  // CTAs whose copies complete on one barrier
+      // One K-type (e = 0) or V-type (e = 1) tile of key tile kt into dst.
+      auto load_tile = [&](uint8_t* dst, const CUtensorMap* map, int e, uint64_t* bar, int h, int kt,
+                           int b) {
+        if constexpr (PAIR) {
+          if (e == 0) {
+            // keys [64 rank, 64 rank + 64) of the tile, all D columns
+#pragma unroll
+            for (int c = 0; c < C::CH; ++c)
+              tma_load_4d_pair(dst + c * C::KROWS * 128, map, leader_addr(bar), c * 64, h,
+                               kt * C::BN + static_cast<int>(rank) * C::KROWS, b, keep);
+          } else {
+            // all keys of the tile, columns [64 rank, 64 rank + 64)
+            tma_load_4d_pair(dst, map, leader_addr(bar), static_cast<int>(rank) * 64, h, kt * C::BN,
+                             b, keep);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < C::CH; ++c)
+            tma_load_4d_hint(dst + c * C::BN * 128, map, bar, c * 64, h, kt * C::BN, b, keep);
+        }
+      };
       uint32_t ctr = 0, q_issued = 0, q_ph = 0;
       bool ok = true;
       int k = 0, pos = 0;
@@ -354,31 +384,14 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
         for (int idx = 0; ok && idx < cnt; ++idx) {
           const int kt = sch.tile(idx);
 #pragma unroll 1
-          for (int u = 0; u < 4; ++u) {
-            const uint32_t slot = ctr % C::NSLOT;
-            const uint32_t ph = (ctr / C::NSLOT) & 1;
-            if (!bwait(&empty[slot], ph ^ 1)) { ok = false; break; }
-            if (mma_cta) mbar_arrive_expect_tx(&full[slot], arm * C::TILE);
-            uint8_t* dst = sRing + slot * C::TILE;
-            if constexpr (PAIR) {
-              if (u < 2) {
-                // K, tK: keys [64 rank, 64 rank + 64) of the tile, all D columns
-#pragma unroll
-                for (int c = 0; c < C::CH; ++c)
-                  tma_load_4d_pair(dst + c * C::KROWS * 128, kv_maps[u], leader_addr(&full[slot]),
-                                   c * 64, w.h, kt * C::BN + static_cast<int>(rank) * C::KROWS, w.b,
-                                   keep);
-              } else {
-                // V, tV: all keys of the tile, columns [64 rank, 64 rank + 64)
-                tma_load_4d_pair(dst, kv_maps[u], leader_addr(&full[slot]),
-                                 static_cast<int>(rank) * 64, w.h, kt * C::BN, w.b, keep);
-              }
-            } else {
-#pragma unroll
-              for (int c = 0; c < C::CH; ++c)
-                tma_load_4d_hint(dst + c * C::BN * 128, kv_maps[u], &full[slot], c * 64, w.h,
-                                 kt * C::BN, w.b, keep);
-            }
+          for (int e = 0; e < 2; ++e) {
+            const uint32_t el = ctr % C::NP;
+            const uint32_t ph = (ctr / C::NP) & 1;
+            if (!bwait(&empty[el], ph ^ 1)) { ok = false; break; }
+            if (mma_cta) mbar_arrive_expect_tx(&full[el], arm * 2 * C::TILE);
+            uint8_t* dst = sRing + el * 2 * C::TILE;
+            load_tile(dst, maps[e][0], e, &full[el], w.h, kt, w.b);
+            load_tile(dst + C::TILE, maps[e][1], e, &full[el], w.h, kt, w.b);
             ++ctr;
           }
         }
@@ -391,9 +404,9 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
           while (globaltimer_ns() - t0 < 2000000ull) __nanosleep(1000);
         } else {
           // Abort: let every copy already issued land before the CTA exits.
-          for (uint32_t s = 0; s < C::NSLOT && s < ctr; ++s) {
-            const uint32_t last = ctr - 1 - ((ctr - 1 + C::NSLOT - s) % C::NSLOT);
-            mbar_wait_drain(&full[s], (last / C::NSLOT) & 1, 200000000ull);
+          for (uint32_t s = 0; s < C::NP && s < ctr; ++s) {
+            const uint32_t last = ctr - 1 - ((ctr - 1 + C::NP - s) % C::NP);
+            mbar_wait_drain(&full[s], (last / C::NP) & 1, 200000000ull);
           }
           if (q_issued > 0) mbar_wait_drain(q_full, (q_issued - 1) & 1, 200000000ull);
         }
@@ -402,33 +415,39 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
     __syncwarp();
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    // Per key tile g (slots 4g..4g+3 hold K_g, tK_g, tV_g, V_g):
-    //   S_{g+1} = Q K_{g+1}^T        once the softmax has read S_g (s_free)
-    //   T (+)= P_g tV_g,  A (+)= P_g V_g          after P_g (p_full)
-    //   T += U_g V_g                               after U_g (u_full)
-    //   tS'_{g+1} = tQ K_{g+1}^T + Q tK_{g+1}^T
-    // S_{g+1} thus runs while the softmax still works on tile g, and the
-    // softmax computes P_{g+1} while P_g's and U_g's products and tS'_{g+1}
-    // run. tcgen05.mma from one thread execute in order, so tS'_{g+1} (over
-    // the columns of P_g and U_g) follows every read of them.
-    // In a pair only the leader's warp 9 issues; its commits arrive on the
-    // barriers of both CTAs.
+    // Per key tile g, with ring elements KK_j = (K_j, tK_j) and VV_j = (tV_j, V_j):
+    //   C: S_{g+1} = Q K_{g+1}^T        once the softmax has read S_g (s_free)
+    //   A: T (+)= P_g tV_g              after P_g (p_full)
+    //   B: A (+)= P_g V_g
+    //   D: T += U_g V_g                 after U_g (u_full)
+    //   E: tS'_{g+1} = tQ K_{g+1}^T + Q tK_{g+1}^T
+    // C goes first when its inputs are ready (it fills the pipe while the
+    // softmax turns tS'_g into P_g), else after B, else after D. tcgen05.mma
+    // from one thread execute in order, so E (over the columns of P_g and
+    // U_g) follows every read of them. The tensor-core queue is shallow and
+    // the issuing thread waits for room, so each barrier a group depends on
+    // is tested in the middle of the group before it (the `rdy_*` flags):
+    // the test's latency then overlaps MMAs still in flight.
+    // The whole warp runs this loop with identical values in every lane (one
+    // elected lane issues each MMA and commit). In a pair only the leader's
+    // warp 9 issues; its commits arrive on the barriers of both CTAs.
     auto commit_all = [&](uint64_t* bar) {
-      if constexpr (PAIR) {
+      if constexpr (PAIR)
         umma_commit_pair_both(bar);
-      } else {
+      else
         umma_commit(bar);
-      }
     };
-    auto poll = [&](uint64_t* bar, uint32_t parity) -> bool {
-      return PAIR ? mbar_test_wait_cluster(bar, parity) : mbar_test_wait(bar, parity);
+    auto test = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __shfl_sync(0xffffffffu, mbar_test_wait(bar, parity) ? 1 : 0, 0) != 0;
     };
-    if (lane == 0 && mma_cta) {
+    if (mma_cta) {
       const uint32_t idesc_s = idesc_bf16_f32(C::M_MMA, C::BN, 0);
       const uint32_t idesc_v = idesc_bf16_f32(C::M_MMA, D, 1);
       const uint32_t aQ = smem_u32(sQ), aTQ = smem_u32(sTQ), aRing = smem_u32(sRing);
-      auto slot_addr = [&](uint32_t c) { return aRing + (c % C::NSLOT) * C::TILE; };
-      auto slot_ph = [&](uint32_t c) { return (c / C::NSLOT) & 1; };
+      auto el_addr = [&](uint32_t j) { return aRing + (j % C::NP) * 2 * C::TILE; };
+      auto el_ph = [&](uint32_t j) { return (j / C::NP) & 1; };
+      auto el_full = [&](uint32_t j) { return &full[j % C::NP]; };
+      auto el_empty = [&](uint32_t j) { return &empty[j % C::NP]; };
       uint32_t q_ph = 0, p_ph = 0, u_ph = 0, sf_ph = 0;
       bool ok = true;
       int k = 0, pos = 0;
@@ -438,27 +457,22 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
         TileSched sch = make_tile_sched(p.mask, w.qt, C::BMU, C::BN);
         int cnt = sch.count(), idx = 0;
         uint32_t g = 0;
-        // prologue: scores of the first tile
-        ok = bwait(q_full, q_ph);
+        // prologue: scores of the first tile (ring element 0 = KK_0)
+        ok = wwait(q_full, q_ph);
         q_ph ^= 1;
-        if (ok) ok = bwait(&full[0], 0);
+        if (ok) ok = wwait(el_full(0), 0);
         if (ok) {
           tc_fence_after();
-          const uint32_t aK = slot_addr(0);
+          const uint32_t aK = el_addr(0), aTK = aK + C::TILE;
           mma_scores<D, C::BM, C::KROWS, PAIR>(tmem + C::TM_S, aQ, aK, idesc_s, false);
           commit_all(s_full);
-          ok = bwait(&full[1], 0);
-          if (ok) {
-            tc_fence_after();
-            const uint32_t aTK = slot_addr(1);
-            mma_scores<D, C::BM, C::KROWS, PAIR>(tmem + C::TM_TS, aTQ, aK, idesc_s, false);
-            mma_scores<D, C::BM, C::KROWS, PAIR>(tmem + C::TM_TS, aQ, aTK, idesc_s, true);
-            commit_all(ts_full);
-            commit_all(&empty[0]);
-            commit_all(&empty[1]);
-            if (cnt == 1) commit_all(q_empty);
-          }
+          mma_scores<D, C::BM, C::KROWS, PAIR>(tmem + C::TM_TS, aTQ, aK, idesc_s, false);
+          mma_scores<D, C::BM, C::KROWS, PAIR>(tmem + C::TM_TS, aQ, aTK, idesc_s, true);
+          commit_all(ts_full);
+          commit_all(el_empty(0));
+          if (cnt == 1) commit_all(q_empty);
         }
+        bool rdy_s = false;  // s_free(g) and KK_{g+1} seen complete
         while (ok) {
           // the tile after g (same item or the next one)
           bool has_next = true, new_item = false;
@@ -476,35 +490,33 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
               new_item = true;
             }
           }
-          const uint32_t c0 = 4 * g, c1 = 4 * (g + 1);
-          const uint32_t aTV = slot_addr(c0 + 2), aV = slot_addr(c0 + 3);
-          // S_{g+1} goes out as soon as the softmax warps have taken S_g out of
-          // TMEM and K_{g+1} has landed: polled (never waited for) between the
-          // groups of this tile, waited for before tS'_{g+1} if still pending.
-          // A new item's first S waits for its Q there too.
-          bool s_done = !has_next;
-#define AJVP_ISSUE_S()                                                                     \
-  do {                                                                                     \
-    tc_fence_after();                                                                      \
-    mma_scores<D, C::BM, C::KROWS, PAIR>(tmem + C::TM_S, aQ, slot_addr(c1), idesc_s, false);        \
-    commit_all(s_full);                                                                   \
-    AJVP_EV(g, 0);                                                                         \
-    s_done = true;                                                                         \
-  } while (0)
-#define AJVP_POLL_S()                                                                      \
-  do {                                                                                     \
-    if (!s_done && !new_item && poll(s_free, sf_ph) &&                           \
-        poll(&full[c1 % C::NSLOT], slot_ph(c1))) {                               \
-      sf_ph ^= 1;                                                                          \
-      AJVP_ISSUE_S();                                                                      \
-    }                                                                                      \
-  } while (0)
-          AJVP_POLL_S();
-          // T (+)= P_g tV_g, A (+)= P_g V_g
-          if (!bwait(&full[(c0 + 2) % C::NSLOT], slot_ph(c0 + 2))) break;
-          if (!bwait(&full[(c0 + 3) % C::NSLOT], slot_ph(c0 + 3))) break;
-          AJVP_POLL_S();
-          if (!bwait(p_full, p_ph)) break;
+          const uint32_t jv = 2 * g + 1, jk = 2 * g + 2;  // VV_g, KK_{g+1}
+          const uint32_t aTV = el_addr(jv), aV = aTV + C::TILE;
+          const uint32_t aK1 = el_addr(jk), aTK1 = aK1 + C::TILE;
+          bool s_done = !has_next, rdy_p = false, rdy_v = false, rdy_u = false, rdy_k = false;
+          AJVP_EV(g, 14);
+          auto issue_s = [&](auto hook) {
+            tc_fence_after();
+            AJVP_EV(g, 12);
+            mma_scores<D, C::BM, C::KROWS, PAIR, D / 32>(tmem + C::TM_S, aQ, aK1, idesc_s, false, hook);
+            commit_all(s_full);
+            AJVP_EV(g, 0);
+            sf_ph ^= 1;
+            s_done = true;
+            rdy_k = true;
+          };
+          // C, early
+          if (!s_done && !new_item &&
+              (rdy_s || (test(s_free, sf_ph) && test(el_full(jk), el_ph(jk))))) {
+            issue_s([&] {
+              rdy_v = test(el_full(jv), el_ph(jv));
+              rdy_p = test(p_full, p_ph);
+            });
+          }
+          // A, B
+          if (!rdy_v && !wwait(el_full(jv), el_ph(jv))) break;
+          AJVP_EV(g, 15);
+          if (!rdy_p && !wwait(p_full, p_ph)) break;
           p_ph ^= 1;
           AJVP_EV(g, 1);
           tc_fence_after();
@@ -512,51 +524,55 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
 #ifdef AJVP_TRACE
           if (!PAIR && p.trace && blockIdx.x == kTraceCta) commit_all(&obs[0]);
 #endif
-          commit_all(&empty[(c0 + 2) % C::NSLOT]);
-          mma_values_split<C::BN, PAIR>(tmem + C::TM_A, tmem + C::TM_P, aV, idesc_v, idx > 0);
+          bool rdy_c = false;
+          mma_values_split<C::BN, PAIR, 3>(tmem + C::TM_A, tmem + C::TM_P, aV, idesc_v, idx > 0, [&] {
+            rdy_u = test(u_full, u_ph);
+            if (!s_done && !new_item) rdy_c = test(s_free, sf_ph) && test(el_full(jk), el_ph(jk));
+          });
 #ifdef AJVP_TRACE
           if (!PAIR && p.trace && blockIdx.x == kTraceCta) commit_all(&obs[1]);
 #endif
           AJVP_EV(g, 2);
-          AJVP_POLL_S();
-          // T += U_g V_g
-          if (!bwait(u_full, u_ph)) break;
+          // C, after B
+          if (rdy_c) issue_s([&] { if (!rdy_u) rdy_u = test(u_full, u_ph); });
+          // D
+          if (!rdy_u && !wwait(u_full, u_ph)) break;
           u_ph ^= 1;
           AJVP_EV(g, 3);
           tc_fence_after();
-          mma_values_split<C::BN, PAIR>(tmem + C::TM_T, tmem + C::TM_U, aV, idesc_v, true);
+          mma_values_split<C::BN, PAIR, 3>(tmem + C::TM_T, tmem + C::TM_U, aV, idesc_v, true, [&] {
+            if (has_next && !rdy_k) rdy_k = test(el_full(jk), el_ph(jk));
+          });
 #ifdef AJVP_TRACE
           if (!PAIR && p.trace && blockIdx.x == kTraceCta) commit_all(&obs[3]);
 #endif
-          commit_all(&empty[(c0 + 3) % C::NSLOT]);
-          commit_all(uv_done);
+          commit_all(el_empty(jv));
           if (idx == cnt - 1) commit_all(acc_full);
           if (!has_next) break;
+          // C, last resort (and always for a new item's first tile, which
+          // needs the new Q)
           if (!s_done) {
             if (new_item) {
-              if (!bwait(q_full, q_ph)) break;
+              if (!wwait(q_full, q_ph)) break;
               q_ph ^= 1;
             }
-            if (!bwait(s_free, sf_ph)) break;
-            sf_ph ^= 1;
-            if (!bwait(&full[c1 % C::NSLOT], slot_ph(c1))) break;
-            AJVP_ISSUE_S();
+            if (!wwait(s_free, sf_ph)) break;
+            if (!wwait(el_full(jk), el_ph(jk))) break;
+            issue_s(NoHook{});
           }
-          // tS'_{g+1}, over the columns of P_g and U_g (read by the MMAs above)
-          if (!bwait(&full[(c1 + 1) % C::NSLOT], slot_ph(c1 + 1))) break;
+          // E, over the columns of P_g and U_g (read by the MMAs above)
+          if (!rdy_k && !wwait(el_full(jk), el_ph(jk))) break;
           tc_fence_after();
-          {
-            const uint32_t aK = slot_addr(c1), aTK = slot_addr(c1 + 1);
-            mma_scores<D, C::BM, C::KROWS, PAIR>(tmem + C::TM_TS, aTQ, aK, idesc_s, false);
-            mma_scores<D, C::BM, C::KROWS, PAIR>(tmem + C::TM_TS, aQ, aTK, idesc_s, true);
-          }
+          const uint32_t jn = jk + 2;  // KK_{g+2}
+          rdy_s = false;
+          mma_scores<D, C::BM, C::KROWS, PAIR>(tmem + C::TM_TS, aTQ, aK1, idesc_s, false);
+          mma_scores<D, C::BM, C::KROWS, PAIR, D / 32>(tmem + C::TM_TS, aQ, aTK1, idesc_s, true, [&] {
+            rdy_s = test(s_free, sf_ph) && test(el_full(jn), el_ph(jn));
+          });
           commit_all(ts_full);
           AJVP_EV(g, 4);
-          commit_all(&empty[c1 % C::NSLOT]);
-          commit_all(&empty[(c1 + 1) % C::NSLOT]);
+          commit_all(el_empty(jk));
           if (idx2 == cnt2 - 1) commit_all(q_empty);
-#undef AJVP_POLL_S
-#undef AJVP_ISSUE_S
           w = w2;
           sch = sch2;
           cnt = cnt2;
@@ -569,7 +585,7 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
         umma_commit_pair(drain);
       else
         umma_commit(drain);
-      mbar_wait_drain(drain, 0, 1000000000ull);
+      if (lane == 0) mbar_wait_drain(drain, 0, 1000000000ull);
     }
     __syncwarp();
   } else {
@@ -710,9 +726,9 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
           resc = true;
         }
         if (__any_sync(0xffffffffu, resc)) {
-          // Every value MMA of earlier tiles has completed once the previous
-          // tile's U V has (they run in issue order).
-          if (!wwait(uv_done, (g - 1) & 1)) { ok = false; break; }
+          // Every value MMA of earlier tiles has completed once this tile's
+          // tS' has (it is issued after them and they run in issue order).
+          if (!wwait(ts_full, ts_ph)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll 1
           for (int c = 0; c < C::DH / 32; ++c) {
@@ -860,21 +876,15 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
   }
 }
 
-size_t tc_smem_bytes(int d, bool pair) {
-  if (d == 128) return pair ? TcCfg<128, true>::BYTES : TcCfg<128, false>::BYTES;
-  return TcCfg<64, false>::BYTES;
+size_t tc_smem_bytes(int d) {
+  return d == 128 ? TcCfg<128, true>::BYTES : TcCfg<64, false>::BYTES;
 }
 
 cudaError_t tc_prepare(int d) {
-  if (d == 128) {
-    cudaError_t e = cudaFuncSetAttribute(attn_jvp_tc_kernel<128, false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         TcCfg<128, false>::BYTES);
-    if (e != cudaSuccess) return e;
+  if (d == 128)
     return cudaFuncSetAttribute(attn_jvp_tc_kernel<128, true>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 TcCfg<128, true>::BYTES);
-  }
   return cudaFuncSetAttribute(attn_jvp_tc_kernel<64, false>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<64, false>::BYTES);
 }
@@ -907,17 +917,14 @@ int tc_pair_max_clusters(int sm_count) {
   return n;
 }
 
-cudaError_t tc_launch(int d, bool pair, const TcParams& p, int grid, cudaStream_t stream) {
-  if (d == 128 && pair) {
+cudaError_t tc_launch(int d, const TcParams& p, int grid, cudaStream_t stream) {
+  if (d == 128) {
     cudaLaunchConfig_t cfg;
     cudaLaunchAttribute attr;
     pair_config(&cfg, &attr, grid, stream);
     return cudaLaunchKernelEx(&cfg, attn_jvp_tc_kernel<128, true>, p);
   }
-  if (d == 128)
-    attn_jvp_tc_kernel<128, false><<<grid, kTcThreads, TcCfg<128, false>::BYTES, stream>>>(p);
-  else
-    attn_jvp_tc_kernel<64, false><<<grid, kTcThreads, TcCfg<64, false>::BYTES, stream>>>(p);
+  attn_jvp_tc_kernel<64, false><<<grid, kTcThreads, TcCfg<64, false>::BYTES, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -40,12 +40,13 @@ constexpr int kTraceEvents = 16;
 constexpr int kTraceCta = 4;  // a CTA (the leader of a pair) whose first items are mostly full tiles
 #endif
 
-size_t tc_smem_bytes(int d, bool pair);
-cudaError_t tc_prepare(int d);  // sets the dynamic shared-memory limits (once per device)
-// Clusters of two CTAs (the pair kernel, d = 128) that fit on the device at once; 0 if unknown.
+size_t tc_smem_bytes(int d);
+cudaError_t tc_prepare(int d);  // sets the dynamic shared-memory limit (once per device)
+// Clusters of two CTAs (the d = 128 kernel runs on CTA pairs) that fit on the
+// device at once; 0 if unknown.
 int tc_pair_max_clusters(int sm_count);
-// pair: launch the CTA-pair kernel (d = 128 only) with `grid` CTAs, an even number.
-cudaError_t tc_launch(int d, bool pair, const TcParams& p, int grid, cudaStream_t stream);
+// d = 128: `grid` CTAs in clusters of two (an even number); d = 64: single CTAs.
+cudaError_t tc_launch(int d, const TcParams& p, int grid, cudaStream_t stream);
 
 // ---- fp32 CUDA-core kernel ----
 constexpr int kSimtBlockQ = 32;

@@ -192,17 +192,6 @@ int attn_jvp_fwd_noalloc(const attn_jvp_shape* shape,
                          void* o, void* to, float* lse,
                          void* stream);
 
-/*
- * attn_jvp_set_cta_pairs - choose the bf16 kernel for head dim 128: 1 runs it
- * on pairs of CTAs (a cluster of two SMs whose tensor-core MMAs cover 256
- * query rows, each SM holding half of every key/value tile); 0 (the default)
- * runs one CTA per 128 query rows. Both compute the same result (they are
- * the same arithmetic in the same order). Process-wide; affects later calls.
- * Returns the previous setting. A tuning and testing switch with no
- * counterpart in the pages.
- */
-int attn_jvp_set_cta_pairs(int enable);
-
 /* ---- host-side helpers (need no GPU) ---------------------------------- */
 
 /* Number of admissible (query, key) pairs per (batch, head):

@@ -94,11 +94,7 @@ struct TcCfg {
   static_assert(TILE == 16384, "16 KB tiles");
   static constexpr int DATA = 2 * QBYTES + NP * 2 * TILE;
   static constexpr int XCH = 2 * BM * 4 + 32;     // row statistics [2][BM] floats + flags [2][4]
-#ifdef AJVP_TRACE
-  static constexpr int NBAR = 2 * NP + 9 + 8 + 4;
-#else
   static constexpr int NBAR = 2 * NP + 9 + 8;
-#endif
   static constexpr int BYTES = 1024 + DATA + XCH + NBAR * 8 + 16;
   static constexpr int ARRIVALS = PAIR ? 16 : 8;  // softmax warps arriving on s_free, p_full, u_full
   static constexpr int HALF = BN / 2;             // key columns per softmax warpgroup
@@ -231,14 +227,15 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
   uint64_t* s_free = bars + 2 * C::NP + 8;
   uint64_t* xa = bars + 2 * C::NP + 9;   // [4] row-statistics exchange, first half
   uint64_t* xb = bars + 2 * C::NP + 13;  // [4] second half
-#ifdef AJVP_TRACE
-  uint64_t* obs = bars + 2 * C::NP + 17;  // [4] MMA-group completion, watched by the observer ([2] unused)
-#endif
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+#ifdef AJVP_TRACE
+  const long long trace_c0 = clock64();
+  const unsigned long long trace_t0 = globaltimer_ns();
+#endif
   // Work is distributed over units: single CTAs, or CTA pairs (clusters of 2).
   const int G = PAIR ? gridDim.x / 2 : gridDim.x;
   const int cta = PAIR ? blockIdx.x / 2 : blockIdx.x;
@@ -280,9 +277,6 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
       mbar_init(&xb[i], 64);
       xflags[i] = 0;
       xflags[4 + i] = 0;
-#ifdef AJVP_TRACE
-      mbar_init(&obs[i], 1);
-#endif
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -304,25 +298,13 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-#ifdef AJVP_TRACE
-  if (!PAIR && warp == 8 && lane == 1 && p.trace && blockIdx.x == kTraceCta) {
-    // observer: completion clocks of P tV, P V and U V of each tile (events
-    // 10, 11, 13; S may complete before or after them and is not observed)
-    for (int g = 0; g < kTraceTiles; ++g) {
-      for (int i = 0; i < 4; ++i) {
-        if (i == 2) continue;
-        if (!mbar_wait_drain(&obs[i], g & 1, 2000000000ull)) { g = kTraceTiles; break; }
-        p.trace[g * kTraceEvents + 10 + i] = static_cast<long long>(clock64());
-      }
-    }
-  }
-#endif
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     // Ring elements in order of first use: per key tile j, (K_j, tK_j) then
     // (tV_j, V_j). In a pair both CTAs load their halves; the copies complete
     // on the leader's barriers, which only the leader's producer arms (for both).
-    if (lane == 0) {
+    // The whole warp runs the loop; one elected lane issues each copy.
+    {
       tma_prefetch_desc(&p.map_q);
       tma_prefetch_desc(&p.map_k);
       tma_prefetch_desc(&p.map_v);
@@ -335,7 +317,8 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
       const uint32_t arm = PAIR ? 2u : 1u;  // CTAs whose copies complete on one barrier
       // One K-type (e = 0) or V-type (e = 1) tile of key tile kt into dst.
       auto load_tile = [&](uint8_t* dst, const CUtensorMap* map, int e, uint64_t* bar, int h, int kt,
-                           int b) {
+                           int b, bool issue) {
+        if (!issue) return;
         if constexpr (PAIR) {
           if (e == 0) {
             // keys [64 rank, 64 rank + 64) of the tile, all D columns
@@ -361,13 +344,14 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
         ++k;
         const WorkItem w = decode_item(p, pos);
         if (q_issued > 0) {
-          if (!bwait(q_empty, q_ph)) { ok = false; break; }
+          if (!wwait(q_empty, q_ph)) { ok = false; break; }
           q_ph ^= 1;
         }
-        if (mma_cta) mbar_arrive_expect_tx(q_full, arm * 2 * C::QBYTES);
         const int q_row = w.qt * C::BMU + static_cast<int>(rank) * C::BM;
+        const bool issue_q = elect_one();
+        if (issue_q && mma_cta) mbar_arrive_expect_tx(q_full, arm * 2 * C::QBYTES);
 #pragma unroll
-        for (int c = 0; c < C::CH; ++c) {
+        for (int c = 0; c < C::CH && issue_q; ++c) {
           if constexpr (PAIR) {
             tma_load_4d_pair(sQ + c * C::BM * 128, &p.map_q, leader_addr(q_full), c * 64, w.h, q_row,
                              w.b, once);
@@ -387,11 +371,12 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
           for (int e = 0; e < 2; ++e) {
             const uint32_t el = ctr % C::NP;
             const uint32_t ph = (ctr / C::NP) & 1;
-            if (!bwait(&empty[el], ph ^ 1)) { ok = false; break; }
-            if (mma_cta) mbar_arrive_expect_tx(&full[el], arm * 2 * C::TILE);
+            if (!wwait(&empty[el], ph ^ 1)) { ok = false; break; }
             uint8_t* dst = sRing + el * 2 * C::TILE;
-            load_tile(dst, maps[e][0], e, &full[el], w.h, kt, w.b);
-            load_tile(dst + C::TILE, maps[e][1], e, &full[el], w.h, kt, w.b);
+            const bool issue = elect_one();
+            if (issue && mma_cta) mbar_arrive_expect_tx(&full[el], arm * 2 * C::TILE);
+            load_tile(dst, maps[e][0], e, &full[el], w.h, kt, w.b, issue);
+            load_tile(dst + C::TILE, maps[e][1], e, &full[el], w.h, kt, w.b, issue);
             ++ctr;
           }
         }
@@ -402,7 +387,7 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
           // them by time (they depend on nothing but memory) before exiting.
           const uint64_t t0 = globaltimer_ns();
           while (globaltimer_ns() - t0 < 2000000ull) __nanosleep(1000);
-        } else {
+        } else if (lane == 0) {
           // Abort: let every copy already issued land before the CTA exits.
           for (uint32_t s = 0; s < C::NP && s < ctr; ++s) {
             const uint32_t last = ctr - 1 - ((ctr - 1 + C::NP - s) % C::NP);
@@ -521,17 +506,11 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
           AJVP_EV(g, 1);
           tc_fence_after();
           mma_values_split<C::BN, PAIR>(tmem + C::TM_T, tmem + C::TM_P, aTV, idesc_v, idx > 0);
-#ifdef AJVP_TRACE
-          if (!PAIR && p.trace && blockIdx.x == kTraceCta) commit_all(&obs[0]);
-#endif
           bool rdy_c = false;
           mma_values_split<C::BN, PAIR, 3>(tmem + C::TM_A, tmem + C::TM_P, aV, idesc_v, idx > 0, [&] {
             rdy_u = test(u_full, u_ph);
             if (!s_done && !new_item) rdy_c = test(s_free, sf_ph) && test(el_full(jk), el_ph(jk));
           });
-#ifdef AJVP_TRACE
-          if (!PAIR && p.trace && blockIdx.x == kTraceCta) commit_all(&obs[1]);
-#endif
           AJVP_EV(g, 2);
           // C, after B
           if (rdy_c) issue_s([&] { if (!rdy_u) rdy_u = test(u_full, u_ph); });
@@ -543,9 +522,6 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
           mma_values_split<C::BN, PAIR, 3>(tmem + C::TM_T, tmem + C::TM_U, aV, idesc_v, true, [&] {
             if (has_next && !rdy_k) rdy_k = test(el_full(jk), el_ph(jk));
           });
-#ifdef AJVP_TRACE
-          if (!PAIR && p.trace && blockIdx.x == kTraceCta) commit_all(&obs[3]);
-#endif
           commit_all(el_empty(jv));
           if (idx == cnt - 1) commit_all(acc_full);
           if (!has_next) break;
@@ -863,6 +839,14 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
     tc_fence_before();
   }
 
+#ifdef AJVP_TRACE
+  // per CTA: SM cycles and nanoseconds from start to here (after every role)
+  if (p.trace && threadIdx.x == 0) {
+    p.trace[kTraceTiles * kTraceEvents + 2 * blockIdx.x] = clock64() - trace_c0;
+    p.trace[kTraceTiles * kTraceEvents + 2 * blockIdx.x + 1] =
+        static_cast<long long>(globaltimer_ns() - trace_t0);
+  }
+#endif
   if constexpr (PAIR) {
     // Neither CTA leaves (or frees its TMEM) while the leader's MMAs may still
     // read the other's shared or tensor memory.

@@ -371,7 +371,7 @@ def run_gpu(args):
                 "peak_source": f"{peak_src} bf16 dense burst",
                 "sustained_peak": float(peaks.get("bf16_tflops_sustained",
                                                   FALLBACK_PEAKS["bf16_tflops_sustained"])),
-                "kernel": "attn_jvp_tc_kernel<128>" if d == 128 else "attn_jvp_tc_kernel<64>",
+                "kernel": "attn_jvp_tc_kernel<128, true> (CTA pairs)" if d == 128 else "attn_jvp_tc_kernel<64, false>",
                 "flops_per_launch": flops, "avg_launch_ms": avg_launch_ms}
     cpu = None
     if world == 1 and not args.no_cpu_baseline:

@@ -34,6 +34,12 @@ diffusion": causal over temporal blocks, full attention inside a block):
 L = n c and a query in chunk j sees keys in chunks <= j.
 Attention inside a chunk is full (bidirectional).
 
+General masks (App. B: the kernel takes masks as query groups with admissible
+key ranges): a table of groups, each a run of consecutive query rows that
+share an admissible key set made of at most two key ranges. The groups cover
+the rows [0, L) in order; group g holds rows [row_end of g-1, row_end of g)
+(0 for the first) and admits keys [k0_begin, k0_end) and [k1_begin, k1_end).
+
 Every function here is pinned by tests/test_oracle_pins.py against values
 that do not come from this file: finite differences, an autodiff JVP of the
 library softmax attention, hand-derived closed forms, hand-written masks,
@@ -48,6 +54,9 @@ import numpy as np
 
 TEACHER_FORCING = 0
 BLOCK_CAUSAL = 1
+
+# One row group: (row_end, k0_begin, k0_end, k1_begin, k1_end).
+Group = Tuple[int, int, int, int, int]
 
 
 def seq_len(mode: int, chunk_tokens: int, n_chunks: int) -> int:
@@ -74,6 +83,40 @@ def allowed(mode: int, c: int, n: int, i, j) -> np.ndarray:
     noisy_q_clean_k = (~i_clean) & j_clean & (cj < ci)
     noisy_q_noisy_k = (~i_clean) & (~j_clean) & (cj == ci)
     return clean_q | noisy_q_clean_k | noisy_q_noisy_k
+
+
+def allowed_groups(groups: Sequence[Group], i, j) -> np.ndarray:
+    """Mask predicate of a group table: True where query row i may attend to
+    key j (`i` and `j` broadcast against each other)."""
+    i = np.asarray(i, dtype=np.int64)
+    j = np.asarray(j, dtype=np.int64)
+    g = np.asarray(groups, dtype=np.int64).reshape(-1, 5)
+    # the group of row i: the first whose row_end exceeds i
+    gi = np.searchsorted(g[:, 0], i, side="right")
+    if np.any(gi >= g.shape[0]):
+        raise ValueError("row beyond the last group")
+    k0b, k0e, k1b, k1e = (g[gi, c] for c in range(1, 5))
+    return ((j >= k0b) & (j < k0e)) | ((j >= k1b) & (j < k1e))
+
+
+def group_table(mode: int, c: int, n: int):
+    """The teacher-forcing or block-causal mask written as a group table: one
+    group per chunk of query rows (clean chunks, then noisy chunks)."""
+    nc = n * c
+    if mode == BLOCK_CAUSAL:
+        return [((j + 1) * c, 0, (j + 1) * c, (j + 1) * c, (j + 1) * c) for j in range(n)]
+    if mode != TEACHER_FORCING:
+        raise ValueError(f"unknown mask mode {mode}")
+    clean = [((j + 1) * c, 0, (j + 1) * c, (j + 1) * c, (j + 1) * c) for j in range(n)]
+    noisy = [(nc + (i + 1) * c, 0, i * c, nc + i * c, nc + (i + 1) * c) for i in range(n)]
+    return clean + noisy
+
+
+def mask_matrix_groups(groups: Sequence[Group]) -> np.ndarray:
+    """Explicit [L, L] boolean mask of a group table (small L only)."""
+    L = int(groups[-1][0])
+    t = np.arange(L)
+    return allowed_groups(groups, t[:, None], t[None, :])
 
 
 def mask_matrix(mode: int, c: int, n: int) -> np.ndarray:
@@ -105,11 +148,13 @@ def _as64(x) -> np.ndarray:
 
 def attn_jvp_rows(q, k, v, tq, tk, tv, mode: int, c: int, n: int,
                   scale: Optional[float], rows: Sequence[int],
-                  block: int = 64) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+                  block: int = 64, groups: Optional[Sequence[Group]] = None
+                  ) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
     """O, tO and LSE for the given query rows of ONE (batch, head).
 
-    q..tv are [L, d] (any float type; promoted to float64). Returns
-    O [R, d], tO [R, d], LSE [R] in float64 for R = len(rows)."""
+    q..tv are [L, d] (any float type; promoted to float64). The mask is the
+    group table `groups` if given, else (mode, c, n). Returns O [R, d],
+    tO [R, d], LSE [R] in float64 for R = len(rows)."""
     q, k, v, tq, tk, tv = (_as64(x) for x in (q, k, v, tq, tk, tv))
     L, d = q.shape
     s = (1.0 / math.sqrt(d)) if scale is None else float(scale)
@@ -121,7 +166,10 @@ def attn_jvp_rows(q, k, v, tq, tk, tv, mode: int, c: int, n: int,
     keys = np.arange(L)
     for r0 in range(0, R, block):
         rr = rows[r0:r0 + block]
-        M = allowed(mode, c, n, rr[:, None], keys[None, :])           # [r, L]
+        if groups is not None:
+            M = allowed_groups(groups, rr[:, None], keys[None, :])    # [r, L]
+        else:
+            M = allowed(mode, c, n, rr[:, None], keys[None, :])       # [r, L]
         S = s * (q[rr] @ k.T)                                        # [r, L]
         S = np.where(M, S, -np.inf)
         smax = S.max(axis=1, keepdims=True)                          # finite: A(i) is never empty
@@ -138,12 +186,17 @@ def attn_jvp_rows(q, k, v, tq, tk, tv, mode: int, c: int, n: int,
 
 
 def attn_jvp_dense(q, k, v, tq, tk, tv, mode: int, c: int, n: int,
-                   scale: Optional[float] = None):
+                   scale: Optional[float] = None,
+                   groups: Optional[Sequence[Group]] = None):
     """Full outputs for [B, L, H, d] inputs: O, tO [B, L, H, d] and LSE
-    [B, H, L], all float64 numpy."""
+    [B, H, L], all float64 numpy. The mask is the group table `groups` if
+    given, else (mode, c, n)."""
     q, k, v, tq, tk, tv = (_as64(x) for x in (q, k, v, tq, tk, tv))
     B, L, H, d = q.shape
-    if L != seq_len(mode, c, n):
+    if groups is not None:
+        if L != int(groups[-1][0]):
+            raise ValueError("L does not match the group table")
+    elif L != seq_len(mode, c, n):
         raise ValueError("L does not match the mask (mode, chunk_tokens, n_chunks)")
     O = np.empty((B, L, H, d))
     tO = np.empty((B, L, H, d))
@@ -153,7 +206,7 @@ def attn_jvp_dense(q, k, v, tq, tk, tv, mode: int, c: int, n: int,
         for h in range(H):
             o_, to_, l_ = attn_jvp_rows(q[b, :, h], k[b, :, h], v[b, :, h],
                                         tq[b, :, h], tk[b, :, h], tv[b, :, h],
-                                        mode, c, n, scale, allrows)
+                                        mode, c, n, scale, allrows, groups=groups)
             O[b, :, h] = o_
             tO[b, :, h] = to_
             lse[b, h] = l_

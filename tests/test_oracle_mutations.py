@@ -32,12 +32,15 @@ def _allowed_block_causal_strict(mode, c, n, i, j):
 
 
 def _rows_variant(kind):
-    def rows(q, k, v, tq, tk, tv, mode, c, n, scale, rows, block=64):
+    def rows(q, k, v, tq, tk, tv, mode, c, n, scale, rows, block=64, groups=None):
         q, k, v, tq, tk, tv = (orc._as64(x) for x in (q, k, v, tq, tk, tv))
         L, d = q.shape
         s = (1.0 / math.sqrt(d)) if scale is None else float(scale)
         rr = np.asarray(rows, dtype=np.int64)
-        M = orc.allowed(mode, c, n, rr[:, None], np.arange(L)[None, :])
+        if groups is not None:
+            M = orc.allowed_groups(groups, rr[:, None], np.arange(L)[None, :])
+        else:
+            M = orc.allowed(mode, c, n, rr[:, None], np.arange(L)[None, :])
         S = np.where(M, s * (q[rr] @ k.T), -np.inf)
         lse = np.logaddexp.reduce(S, axis=1)
         P = np.exp(S - lse[:, None])
@@ -123,3 +126,50 @@ def test_jvp_mistakes_are_caught(monkeypatch, kind):
 def test_correct_rewrite_is_not_flagged(monkeypatch):
     # the same formula written independently passes all pins (no false alarms)
     assert _caught(monkeypatch, "attn_jvp_rows", _rows_variant("none")) == 0
+
+
+def _groups_row_boundary_off_by_one(groups, i, j):
+    # mistake: the last row of each group is given the next group's keys
+    i = np.asarray(i, dtype=np.int64)
+    g = np.asarray(groups, dtype=np.int64).reshape(-1, 5)
+    gi = np.minimum(np.searchsorted(g[:, 0], i + 1, side="right"), g.shape[0] - 1)
+    j = np.asarray(j, dtype=np.int64)
+    k0b, k0e, k1b, k1e = (g[gi, c] for c in range(1, 5))
+    return ((j >= k0b) & (j < k0e)) | ((j >= k1b) & (j < k1e))
+
+
+def _groups_end_inclusive(groups, i, j):
+    # mistake: key ranges taken as closed intervals
+    i = np.asarray(i, dtype=np.int64)
+    g = np.asarray(groups, dtype=np.int64).reshape(-1, 5)
+    gi = np.searchsorted(g[:, 0], i, side="right")
+    j = np.asarray(j, dtype=np.int64)
+    k0b, k0e, k1b, k1e = (g[gi, c] for c in range(1, 5))
+    return ((j >= k0b) & (j <= k0e)) | ((j >= k1b) & (j <= k1e))
+
+
+GROUP_PIN_CHECKS = [
+    lambda: pins.test_group_mask_matches_hand_written(),
+    lambda: pins.test_groups_against_torch_autodiff(),
+]
+for _m in (TF, orc.BLOCK_CAUSAL):
+    for _c, _n in ((2, 3), (5, 4)):
+        GROUP_PIN_CHECKS.append(
+            lambda m=_m, c=_c, n=_n: pins.test_group_table_of_each_mode_gives_its_mask(m, c, n))
+
+
+@pytest.mark.parametrize("mutant", [_groups_row_boundary_off_by_one, _groups_end_inclusive])
+def test_group_mask_mistakes_are_caught(monkeypatch, mutant):
+    monkeypatch.setattr(orc, "allowed_groups", mutant)
+    failures = 0
+    for check in GROUP_PIN_CHECKS:
+        try:
+            check()
+        except (AssertionError, IndexError):
+            failures += 1
+    assert failures > 0
+
+
+def test_group_pins_pass_unmutated():
+    for check in GROUP_PIN_CHECKS:
+        check()

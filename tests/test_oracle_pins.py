@@ -51,6 +51,60 @@ def test_mask_matches_hand_written(fname, mode, c, n):
     assert np.array_equal(orc.mask_matrix(mode, c, n), _read_mask(fname))
 
 
+GROUPS_EXAMPLE = [(2, 0, 3, 6, 8), (5, 1, 2, 4, 6), (8, 5, 8, 8, 8)]
+
+
+def test_group_mask_matches_hand_written():
+    assert np.array_equal(orc.mask_matrix_groups(GROUPS_EXAMPLE),
+                          _read_mask("mask_groups_example.txt"))
+
+
+@pytest.mark.parametrize("mode", [TF, BC])
+@pytest.mark.parametrize("c,n", [(1, 1), (2, 3), (3, 1), (5, 4)])
+def test_group_table_of_each_mode_gives_its_mask(mode, c, n):
+    # two restatements of the same mask (chunk rule vs. per-group key ranges)
+    assert np.array_equal(orc.mask_matrix_groups(orc.group_table(mode, c, n)),
+                          orc.mask_matrix(mode, c, n))
+
+
+def test_groups_path_matches_mode_path_numerically():
+    rng = np.random.default_rng(5)
+    c, n, d = 3, 3, 8
+    L = 2 * n * c
+    x = [rng.standard_normal((1, L, 2, d)) for _ in range(6)]
+    a = orc.attn_jvp_dense(*x, TF, c, n)
+    b = orc.attn_jvp_dense(*x, TF, c, n, groups=orc.group_table(TF, c, n))
+    for u, w in zip(a, b):
+        assert np.array_equal(u, w)
+
+
+def test_groups_against_torch_autodiff():
+    # JVP of the library's softmax attention (MATH backend) under the
+    # hand-written group mask
+    import torch
+    from torch.func import jvp
+    rng = np.random.default_rng(11)
+    M = _read_mask("mask_groups_example.txt")
+    L, d = M.shape[0], 4
+    q, k, v, tq, tk, tv = (rng.standard_normal((L, d)) for _ in range(6))
+    O, tO, lse = orc.attn_jvp_rows(q, k, v, tq, tk, tv, TF, 1, 1, None, np.arange(L),
+                                   groups=GROUPS_EXAMPLE)
+    mask = torch.from_numpy(M)
+
+    def f(qq, kk, vv):
+        with torch.nn.attention.sdpa_kernel(torch.nn.attention.SDPBackend.MATH):
+            return torch.nn.functional.scaled_dot_product_attention(
+                qq[None, None], kk[None, None], vv[None, None], attn_mask=mask)[0, 0]
+
+    T = lambda a: torch.from_numpy(a)
+    o_ref, to_ref = jvp(f, (T(q), T(k), T(v)), (T(tq), T(tk), T(tv)))
+    assert np.allclose(O, o_ref.numpy(), atol=1e-12, rtol=1e-10)
+    assert np.allclose(tO, to_ref.numpy(), atol=1e-12, rtol=1e-10)
+    s = 1.0 / math.sqrt(d)
+    S = np.where(M, s * q @ k.T, -np.inf)
+    assert np.allclose(lse, np.log(np.exp(S).sum(axis=1)), atol=1e-12)
+
+
 @pytest.mark.parametrize("c", [1, 2, 3, 5, 16])
 @pytest.mark.parametrize("n", [1, 2, 3, 7])
 def test_pair_count_closed_form(c, n):

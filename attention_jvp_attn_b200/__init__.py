@@ -12,7 +12,7 @@ from __future__ import annotations
 
 import ctypes
 import math
-from typing import List, Optional, Tuple
+from typing import List, Optional, Sequence, Tuple
 
 import torch
 
@@ -20,7 +20,7 @@ from . import _abi
 from ._abi import AttnJvpError  # noqa: F401
 from .inputs import BLOCK_CAUSAL, TEACHER_FORCING  # noqa: F401
 
-__all__ = ["attn_jvp", "attn_jvp_host", "sync_status", "unmasked_pairs", "schedule_tiles",
+__all__ = ["attn_jvp", "attn_jvp_groups", "attn_jvp_host", "sync_status", "unmasked_pairs", "schedule_tiles",
            "host_staging_bytes", "AttnJvpError", "TEACHER_FORCING", "BLOCK_CAUSAL"]
 
 _DT = {torch.bfloat16: _abi.DTYPE_BF16, torch.float32: _abi.DTYPE_F32}
@@ -72,6 +72,40 @@ def attn_jvp(q, k, v, tq, tk, tv, mode: int, chunk_tokens: int, n_chunks: int,
                               o.data_ptr(), to.data_ptr(), lse.data_ptr(),
                               _stream_handle(q.device))
     _abi.check(rc, "attn_jvp_fwd")
+    return o, to, lse
+
+
+def attn_jvp_groups(q, k, v, tq, tk, tv, groups: Sequence[Tuple[int, int, int, int, int]],
+                    scale: Optional[float] = None,
+                    out: Optional[Tuple[torch.Tensor, torch.Tensor, torch.Tensor]] = None):
+    """attn_jvp with a general mask: `groups` is a table of
+    (row_end, k0_begin, k0_end, k1_begin, k1_end) row groups in row order, the
+    last ending at L; rows of a group may attend to keys [k0_begin, k0_end)
+    and [k1_begin, k1_end)."""
+    ts = (q, k, v, tq, tk, tv)
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("inputs must be CUDA tensors")
+        if t.shape != q.shape or t.dtype != q.dtype or t.device != q.device:
+            raise ValueError("q, k, v, tq, tk, tv must share shape, dtype and device")
+        if not t.is_contiguous():
+            raise ValueError("inputs must be contiguous [B, L, H, d]")
+    shape = _shape(q, scale)
+    B, L, H, d = q.shape
+    if out is None:
+        o = torch.empty_like(q)
+        to = torch.empty_like(q)
+        lse = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
+    else:
+        o, to, lse = out
+    table = _abi.group_array(groups)
+    lib = _abi.load()
+    with torch.cuda.device(q.device):
+        rc = lib.attn_jvp_fwd_groups(ctypes.byref(shape), q.data_ptr(), k.data_ptr(),
+                                     v.data_ptr(), tq.data_ptr(), tk.data_ptr(), tv.data_ptr(),
+                                     table, len(groups), o.data_ptr(), to.data_ptr(),
+                                     lse.data_ptr(), _stream_handle(q.device))
+    _abi.check(rc, "attn_jvp_fwd_groups")
     return o, to, lse
 
 

@@ -31,6 +31,23 @@ class Mask(ctypes.Structure):
                 ("n_chunks", ctypes.c_int32)]
 
 
+MAX_GROUPS = 512
+
+
+class Group(ctypes.Structure):
+    _fields_ = [("row_end", ctypes.c_int32), ("k0_begin", ctypes.c_int32),
+                ("k0_end", ctypes.c_int32), ("k1_begin", ctypes.c_int32),
+                ("k1_end", ctypes.c_int32)]
+
+
+def group_array(groups):
+    """A ctypes array of Group from (row_end, k0_begin, k0_end, k1_begin, k1_end) tuples."""
+    arr = (Group * max(1, len(groups)))()
+    for i, g in enumerate(groups):
+        arr[i] = Group(*(int(x) for x in g))
+    return arr
+
+
 _lib = None
 _lock = threading.Lock()
 
@@ -71,6 +88,14 @@ def load(path: str = None) -> ctypes.CDLL:
         lib.attn_jvp_fwd_noalloc.argtypes = [ctypes.POINTER(Shape), vp, vp, vp, vp, vp, vp,
                                              Mask, vp, vp, vp, vp]
         lib.attn_jvp_fwd_noalloc.restype = ctypes.c_int
+        lib.attn_jvp_fwd_groups.argtypes = [ctypes.POINTER(Shape), vp, vp, vp, vp, vp, vp,
+                                            ctypes.POINTER(Group), ctypes.c_int32, vp, vp, vp, vp]
+        lib.attn_jvp_fwd_groups.restype = ctypes.c_int
+        lib.attn_jvp_schedule_tiles_groups.argtypes = [
+            ctypes.POINTER(Group), ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+            ctypes.c_int32, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_uint8),
+            ctypes.c_int32]
+        lib.attn_jvp_schedule_tiles_groups.restype = ctypes.c_int32
         lib.attn_jvp_version.argtypes = []
         lib.attn_jvp_version.restype = ctypes.c_int32
         _lib = lib

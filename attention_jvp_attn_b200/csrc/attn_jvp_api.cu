@@ -105,6 +105,40 @@ int validate_mask(const attn_jvp_mask& m, int64_t* L_expected) {
   return ATTN_JVP_OK;
 }
 
+// Shape checks common to both mask forms (L is checked against the mask by the caller).
+int validate_shape(const attn_jvp_shape* s) {
+  if (!s) return ATTN_JVP_ERR_INVALID_ARGUMENT;
+  if (s->B < 1 || s->H < 1 || s->L < 1) return ATTN_JVP_ERR_INVALID_ARGUMENT;
+  if (s->dtype != ATTN_JVP_BF16 && s->dtype != ATTN_JVP_F32) return ATTN_JVP_ERR_UNSUPPORTED;
+  if (s->d != 64 && s->d != 128) return ATTN_JVP_ERR_UNSUPPORTED;
+  if (!(s->scale <= 0.f || std::isfinite(s->scale))) return ATTN_JVP_ERR_INVALID_ARGUMENT;
+  if (s->L > kMaxSeq) return ATTN_JVP_ERR_INVALID_ARGUMENT;
+  if (s->B > 65535 || s->H > 65535) return ATTN_JVP_ERR_INVALID_ARGUMENT;
+  if (s->B * s->H * ((s->L + ajvp::kTcBlockM - 1) / ajvp::kTcBlockM) > int64_t(1) << 31)
+    return ATTN_JVP_ERR_INVALID_ARGUMENT;
+  return ATTN_JVP_OK;
+}
+
+// A group table: 1..ATTN_JVP_MAX_GROUPS groups whose row_end increase to L,
+// each with 0 <= k0_begin <= k0_end <= k1_begin <= k1_end <= L and at least
+// one admissible key.
+int validate_groups(const attn_jvp_shape* s, const attn_jvp_group* g, int32_t n) {
+  if (!g || n < 1) return ATTN_JVP_ERR_INVALID_ARGUMENT;
+  if (n > ATTN_JVP_MAX_GROUPS) return ATTN_JVP_ERR_UNSUPPORTED;
+  int64_t prev = 0;
+  for (int32_t i = 0; i < n; ++i) {
+    const attn_jvp_group& x = g[i];
+    if (x.row_end <= prev) return ATTN_JVP_ERR_INVALID_ARGUMENT;
+    if (x.k0_begin < 0 || x.k0_begin > x.k0_end || x.k0_end > x.k1_begin ||
+        x.k1_begin > x.k1_end || x.k1_end > s->L)
+      return ATTN_JVP_ERR_INVALID_ARGUMENT;
+    if (x.k0_end - x.k0_begin + x.k1_end - x.k1_begin <= 0) return ATTN_JVP_ERR_INVALID_ARGUMENT;
+    prev = x.row_end;
+  }
+  if (prev != s->L) return ATTN_JVP_ERR_INVALID_ARGUMENT;
+  return ATTN_JVP_OK;
+}
+
 int validate(const attn_jvp_shape* s, attn_jvp_mask mask) {
   if (!s) return ATTN_JVP_ERR_INVALID_ARGUMENT;
   if (s->B < 1 || s->H < 1 || s->L < 1) return ATTN_JVP_ERR_INVALID_ARGUMENT;
@@ -145,7 +179,37 @@ MaskSpec mask_spec(attn_jvp_mask m, int64_t L) {
   ms.c = m.chunk_tokens;
   ms.n = m.n_chunks;
   ms.L = static_cast<int>(L);
+  ms.n_groups = 0;
+  ms.groups = nullptr;
   return ms;
+}
+
+// A validated group table in the kernels' form (host copy, for the launch).
+struct GroupTable {
+  ajvp::GroupRange g[ajvp::kMaxGroups];
+  int n = 0;
+};
+
+MaskSpec groups_spec(const attn_jvp_group* groups, int32_t n, int64_t L, GroupTable* t) {
+  for (int32_t i = 0; i < n; ++i)
+    t->g[i] = ajvp::GroupRange{groups[i].row_end, groups[i].k0_begin, groups[i].k0_end,
+                               groups[i].k1_begin, groups[i].k1_end};
+  t->n = n;
+  MaskSpec ms;
+  ms.mode = ajvp::kModeGroups;
+  ms.c = ms.n = 0;
+  ms.L = static_cast<int>(L);
+  ms.n_groups = n;
+  ms.groups = t->g;
+  return ms;
+}
+
+// The mask as the kernels' parameters carry it: a table (if any) is copied in.
+void set_mask(MaskSpec* dst, ajvp::GroupRange* dst_groups, const MaskSpec& ms) {
+  *dst = ms;
+  if (ms.mode == ajvp::kModeGroups)
+    std::memcpy(dst_groups, ms.groups, sizeof(ajvp::GroupRange) * ms.n_groups);
+  dst->groups = nullptr;  // the kernels point it at their own parameter copy
 }
 
 // Query row blocks (of `bm` rows) of one head, most key tiles first (stable among equals).
@@ -162,7 +226,7 @@ int fill_order(const MaskSpec& ms, int n_qtiles, int bm, uint16_t* order) {
 }
 
 int launch_bf16(DeviceState* st, const attn_jvp_shape* s, const void* q, const void* k,
-                const void* v, const void* tq, const void* tk, const void* tv, attn_jvp_mask mask,
+                const void* v, const void* tq, const void* tk, const void* tv, const MaskSpec& ms,
                 void* o, void* to, float* lse, cudaStream_t stream) {
   static thread_local ajvp::TcParams p;  // large (order table): not on the stack
   std::memset(&p, 0, offsetof(ajvp::TcParams, order));
@@ -187,11 +251,11 @@ int launch_bf16(DeviceState* st, const attn_jvp_shape* s, const void* q, const v
   p.L = static_cast<int>(s->L);
   p.n_qtiles = static_cast<int>((s->L + bmu - 1) / bmu);
   p.n_items = p.B * p.H * p.n_qtiles;
-  p.mask = mask_spec(mask, s->L);
+  set_mask(&p.mask, p.groups, ms);
   const float sc = softmax_scale(s);
   p.scale = sc;
   p.scale_log2 = sc * 1.4426950408889634f;
-  p.order_len = fill_order(p.mask, p.n_qtiles, bmu, p.order);
+  p.order_len = fill_order(ms, p.n_qtiles, bmu, p.order);
 #ifdef AJVP_TRACE
   p.trace = g_trace;
 #endif
@@ -203,9 +267,9 @@ int launch_bf16(DeviceState* st, const attn_jvp_shape* s, const void* q, const v
 }
 
 int launch_f32(const attn_jvp_shape* s, const void* q, const void* k, const void* v,
-               const void* tq, const void* tk, const void* tv, attn_jvp_mask mask, void* o,
+               const void* tq, const void* tk, const void* tv, const MaskSpec& ms, void* o,
                void* to, float* lse, cudaStream_t stream) {
-  ajvp::SimtParams p;
+  static thread_local ajvp::SimtParams p;  // large (group table): not on the stack
   p.q = static_cast<const float*>(q);
   p.k = static_cast<const float*>(k);
   p.v = static_cast<const float*>(v);
@@ -218,7 +282,7 @@ int launch_f32(const attn_jvp_shape* s, const void* q, const void* k, const void
   p.B = static_cast<int>(s->B);
   p.H = static_cast<int>(s->H);
   p.L = static_cast<int>(s->L);
-  p.mask = mask_spec(mask, s->L);
+  set_mask(&p.mask, p.groups, ms);
   const float sc = softmax_scale(s);
   p.scale = sc;
   p.scale_log2 = sc * 1.4426950408889634f;
@@ -227,6 +291,23 @@ int launch_f32(const attn_jvp_shape* s, const void* q, const void* k, const void
 }
 
 int64_t round256(int64_t x) { return (x + 255) & ~int64_t(255); }
+
+// Pointer checks and the launch for either dtype (shape and mask validated).
+int run_checked(const attn_jvp_shape* shape, const void* q, const void* k, const void* v,
+                const void* tq, const void* tk, const void* tv, const MaskSpec& ms, void* o,
+                void* to, float* lse, void* stream) {
+  const void* ptrs[9] = {q, k, v, tq, tk, tv, o, to, lse};
+  for (const void* ptr : ptrs)
+    if (!ptr) return ATTN_JVP_ERR_INVALID_ARGUMENT;
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return ATTN_JVP_ERR_MISALIGNED;
+  DeviceState* st = nullptr;
+  const int rc = device_state(&st);
+  if (rc != ATTN_JVP_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (shape->dtype == ATTN_JVP_BF16) return launch_bf16(st, shape, q, k, v, tq, tk, tv, ms, o, to, lse, s);
+  return launch_f32(shape, q, k, v, tq, tk, tv, ms, o, to, lse, s);
+}
 
 // ---- allocation-free variant ---------------------------------------------
 // Scratch of attn_jvp_fwd_noalloc: a file-scope device array (one per device
@@ -301,19 +382,22 @@ extern "C" {
 int attn_jvp_fwd(const attn_jvp_shape* shape, const void* q, const void* k, const void* v,
                  const void* tq, const void* tk, const void* tv, attn_jvp_mask mask, void* o,
                  void* to, float* lse, void* stream) {
-  int rc = validate(shape, mask);
+  const int rc = validate(shape, mask);
   if (rc != ATTN_JVP_OK) return rc;
-  const void* ptrs[9] = {q, k, v, tq, tk, tv, o, to, lse};
-  for (const void* ptr : ptrs)
-    if (!ptr) return ATTN_JVP_ERR_INVALID_ARGUMENT;
-  for (const void* ptr : ptrs)
-    if (!aligned16(ptr)) return ATTN_JVP_ERR_MISALIGNED;
-  DeviceState* st = nullptr;
-  rc = device_state(&st);
+  return run_checked(shape, q, k, v, tq, tk, tv, mask_spec(mask, shape->L), o, to, lse, stream);
+}
+
+int attn_jvp_fwd_groups(const attn_jvp_shape* shape, const void* q, const void* k, const void* v,
+                        const void* tq, const void* tk, const void* tv,
+                        const attn_jvp_group* groups, int32_t n_groups, void* o, void* to,
+                        float* lse, void* stream) {
+  int rc = validate_shape(shape);
   if (rc != ATTN_JVP_OK) return rc;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (shape->dtype == ATTN_JVP_BF16) return launch_bf16(st, shape, q, k, v, tq, tk, tv, mask, o, to, lse, s);
-  return launch_f32(shape, q, k, v, tq, tk, tv, mask, o, to, lse, s);
+  rc = validate_groups(shape, groups, n_groups);
+  if (rc != ATTN_JVP_OK) return rc;
+  static thread_local GroupTable table;
+  const MaskSpec ms = groups_spec(groups, n_groups, shape->L, &table);
+  return run_checked(shape, q, k, v, tq, tk, tv, ms, o, to, lse, stream);
 }
 
 int64_t attn_jvp_host_staging_bytes(const attn_jvp_shape* shape) {
@@ -401,6 +485,25 @@ int64_t attn_jvp_unmasked_pairs(attn_jvp_mask mask) {
   return mask.mode == ATTN_JVP_MASK_TEACHER_FORCING ? tf : tf / 2;
 }
 
+int32_t attn_jvp_schedule_tiles_groups(const attn_jvp_group* groups, int32_t n_groups, int64_t L,
+                                       int32_t block_m, int32_t block_n, int32_t q_tile,
+                                       int32_t* tiles, uint8_t* full, int32_t cap) {
+  attn_jvp_shape shape{1, L, 1, 64, ATTN_JVP_BF16, 0.f};
+  if (L < 1 || L > kMaxSeq || validate_groups(&shape, groups, n_groups) != ATTN_JVP_OK) return -1;
+  if (block_m < 1 || block_n < 1 || q_tile < 0 || cap < 0) return -1;
+  if (int64_t(q_tile) * block_m >= L) return -1;
+  if ((tiles == nullptr || full == nullptr) && cap > 0) return -1;
+  static thread_local GroupTable table;
+  const MaskSpec ms = groups_spec(groups, n_groups, L, &table);
+  const ajvp::TileSched s = ajvp::make_tile_sched(ms, q_tile, block_m, block_n);
+  const int n = s.count();
+  for (int i = 0; i < n && i < cap; ++i) {
+    tiles[i] = s.tile(i);
+    full[i] = s.full(s.tile(i)) ? 1 : 0;
+  }
+  return n;
+}
+
 int32_t attn_jvp_schedule_tiles(attn_jvp_mask mask, int64_t L, int32_t block_m, int32_t block_n,
                                 int32_t q_tile, int32_t* tiles, uint8_t* full, int32_t cap) {
   int64_t Lx = 0;
@@ -447,7 +550,8 @@ int attn_jvp_fwd_noalloc(const attn_jvp_shape* shape, const void* q, const void*
   launch_state.sm_count = st->sm_count;
   launch_state.pair_clusters = st->pair_clusters;
   launch_state.status = st->scratch;
-  rc = launch_bf16(&launch_state, shape, q, k, v, tq, tk, tv, mask, o, to, lse, s);
+  rc = launch_bf16(&launch_state, shape, q, k, v, tq, tk, tv, mask_spec(mask, shape->L), o, to, lse,
+                   s);
   if (rc != ATTN_JVP_OK) return rc;
   if (cudaStreamSynchronize(s) != cudaSuccess) {
     cudaGetLastError();

@@ -28,7 +28,7 @@ struct SimtCfg {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kSimtThreads) attn_jvp_simt_kernel(const SimtParams p) {
+__global__ void __launch_bounds__(kSimtThreads) attn_jvp_simt_kernel(const __grid_constant__ SimtParams p) {
   using C = SimtCfg<D>;
   extern __shared__ float sm[];
   float* sK = sm;
@@ -39,6 +39,8 @@ __global__ void __launch_bounds__(kSimtThreads) attn_jvp_simt_kernel(const SimtP
   float* sTQ = sQ + C::BQ * D;
 
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  MaskSpec mask = p.mask;  // with the group table (if any) from this launch's parameters
+  mask.groups = p.groups;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int L = p.L, H = p.H;
   const size_t rs = static_cast<size_t>(H) * D;  // row stride of [B, L, H, d]
@@ -61,10 +63,10 @@ __global__ void __launch_bounds__(kSimtThreads) attn_jvp_simt_kernel(const SimtP
     ds[i] = 0.f;
 #pragma unroll
     for (int u = 0; u < C::CPL; ++u) A[i][u] = T[i][u] = 0.f;
-    rr[i] = row_range(p.mask, qt * C::BQ + warp * C::RPW + i);
+    rr[i] = row_range(mask, qt * C::BQ + warp * C::RPW + i);
   }
 
-  const TileSched sch = make_tile_sched(p.mask, qt, C::BQ, C::BK);
+  const TileSched sch = make_tile_sched(mask, qt, C::BQ, C::BK);
   const int cnt = sch.count();
   for (int idx = 0; idx < cnt; ++idx) {
     const int k0 = sch.tile(idx) * C::BK;

@@ -240,6 +240,9 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
   const int G = PAIR ? gridDim.x / 2 : gridDim.x;
   const int cta = PAIR ? blockIdx.x / 2 : blockIdx.x;
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;  // 0: issues the MMAs
+  // The mask, with a group table (if any) read from this launch's parameters.
+  MaskSpec mask = p.mask;
+  mask.groups = p.groups;
   const bool mma_cta = rank == 0;
   // Barriers the leader waits on and other threads (of either CTA) arrive on.
   auto leader_addr = [&](uint64_t* bar) -> uint32_t {
@@ -363,7 +366,7 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
           }
         }
         ++q_issued;
-        const TileSched sch = make_tile_sched(p.mask, w.qt, C::BMU, C::BN);
+        const TileSched sch = make_tile_sched(mask, w.qt, C::BMU, C::BN);
         const int cnt = sch.count();
         for (int idx = 0; ok && idx < cnt; ++idx) {
           const int kt = sch.tile(idx);
@@ -439,7 +442,7 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
       if (next_item(p, cta, G, k, pos)) {
         ++k;
         WorkItem w = decode_item(p, pos);
-        TileSched sch = make_tile_sched(p.mask, w.qt, C::BMU, C::BN);
+        TileSched sch = make_tile_sched(mask, w.qt, C::BMU, C::BN);
         int cnt = sch.count(), idx = 0;
         uint32_t g = 0;
         // prologue: scores of the first tile (ring element 0 = KK_0)
@@ -469,7 +472,7 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
             if (has_next) {
               ++k;
               w2 = decode_item(p, pos);
-              sch2 = make_tile_sched(p.mask, w2.qt, C::BMU, C::BN);
+              sch2 = make_tile_sched(mask, w2.qt, C::BMU, C::BN);
               cnt2 = sch2.count();
               idx2 = 0;
               new_item = true;
@@ -639,8 +642,8 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
       ++k;
       const WorkItem w = decode_item(p, pos);
       const int t = w.qt * C::BMU + static_cast<int>(rank) * C::BM + row;  // this thread's query row
-      const RowRange rr = row_range(p.mask, t);
-      const TileSched sch = make_tile_sched(p.mask, w.qt, C::BMU, C::BN);
+      const RowRange rr = row_range(mask, t);
+      const TileSched sch = make_tile_sched(mask, w.qt, C::BMU, C::BN);
       const int cnt = sch.count();
       float m_use = -INFINITY, l = 0.f, dsum = 0.f;
       for (int idx = 0; idx < cnt; ++idx, ++g) {
@@ -656,14 +659,16 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
         tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
         tmem_wait_ld();
         if (!full_tile) {
-          // admissible local columns of this row in this half tile, [0, e1) U
+          // admissible local columns of this row in this half tile, [s1, e1) U
           // [s2, e2), as 32-bit column masks
+          const int s1 = min(max(rr.a0 - k0, 0), C::HALF);
           const int e1 = min(max(rr.a1 - k0, 0), C::HALF);
           const int s2 = min(max(rr.b0 - k0, 0), C::HALF);
           const int e2 = min(max(rr.b1 - k0, 0), C::HALF);
 #pragma unroll
           for (int q = 0; q < C::HALF / 32; ++q) {
-            const uint32_t m = low_bits(e1 - 32 * q) | (low_bits(e2 - 32 * q) & ~low_bits(s2 - 32 * q));
+            const uint32_t m = (low_bits(e1 - 32 * q) & ~low_bits(s1 - 32 * q)) |
+                               (low_bits(e2 - 32 * q) & ~low_bits(s2 - 32 * q));
 #pragma unroll
             for (int j = 0; j < 32; ++j)
               if (!((m >> j) & 1u)) sr[32 * q + j] = __float_as_uint(-INFINITY);

@@ -29,9 +29,10 @@ struct TcParams {
   float scale;       // s
   int order_len;     // n_qtiles if `order` is filled, else 0 (reverse index order)
 #ifdef AJVP_TRACE
-  long long* trace;  // per-tile event clocks of CTA 0 (trace builds only)
+  long long* trace;  // per-tile event clocks of one CTA (trace builds only)
 #endif
   uint16_t order[kMaxOrder];
+  GroupRange groups[kMaxGroups];  // mask.mode == kModeGroups: the row groups (mask.n_groups)
 };
 
 #ifdef AJVP_TRACE
@@ -59,6 +60,7 @@ struct SimtParams {
   int B, H, L;
   MaskSpec mask;
   float scale_log2, scale;
+  GroupRange groups[kMaxGroups];  // mask.mode == kModeGroups: the row groups (mask.n_groups)
 };
 
 size_t simt_smem_bytes(int d);

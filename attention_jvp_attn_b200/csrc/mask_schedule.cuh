@@ -11,10 +11,14 @@
 //     clean query in chunk j:  keys [0, (j+1) c)
 //     noisy query in chunk i:  keys [0, i c)  U  [nc + i c, nc + (i+1) c)
 //   block causal: L = n c, query in chunk j: keys [0, (j+1) c)
-// Every row's admissible set is [0, a1) U [b0, b1) (second part possibly
-// empty). All first parts lie in [0, nc), all second parts in [nc, 2nc), so a
-// group of rows has union [0, max a1) U [min b0, max b1) and intersection
-// [0, min a1) U (common b-range if all rows share one noisy chunk).
+//   groups (the general form of the same page's App. B: query groups with
+//     admissible key ranges): a table of row groups in order; group g holds
+//     rows [row_end of g-1, row_end of g) and admits keys [a0, a1) U [b0, b1).
+// Every row's admissible set is [a0, a1) U [b0, b1) (either part possibly
+// empty; a1 <= b0). A block of rows is scheduled over the union
+// [min a0, max a1) U [min b0, max b1) (a gap inside either part is visited
+// and masked); a key tile is "full" inside the intersection
+// [max a0, min a1) U (the b-range, if every row has the same one).
 #pragma once
 
 #include <cstdint>
@@ -27,22 +31,53 @@
 
 namespace ajvp {
 
-enum : int { kModeTeacherForcing = 0, kModeBlockCausal = 1 };
+enum : int { kModeTeacherForcing = 0, kModeBlockCausal = 1, kModeGroups = 2 };
+
+// One row group of a general mask: rows up to row_end (exclusive) since the
+// previous group, keys [a0, a1) U [b0, b1).
+struct GroupRange {
+  int row_end, a0, a1, b0, b1;
+};
+constexpr int kMaxGroups = 512;
 
 struct MaskSpec {
   int mode;
   int c;  // chunk tokens
   int n;  // chunks
   int L;  // sequence length
+  int n_groups;               // kModeGroups: table length
+  const GroupRange* groups;   // kModeGroups: the table (host or device address)
 };
 
-// Admissible keys of one query row: [0, a1) U [b0, b1).
+// Admissible keys of one query row: [a0, a1) U [b0, b1).
 struct RowRange {
-  int a1, b0, b1;
+  int a0, a1, b0, b1;
 };
+
+// Index of the group holding row t: the first with row_end > t.
+AJVP_HD int group_of(const MaskSpec& m, int t) {
+  int lo = 0, hi = m.n_groups - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (m.groups[mid].row_end > t)
+      hi = mid;
+    else
+      lo = mid + 1;
+  }
+  return lo;
+}
 
 AJVP_HD RowRange row_range(const MaskSpec& m, int t) {
   RowRange r;
+  r.a0 = 0;
+  if (m.mode == kModeGroups) {
+    const GroupRange g = m.groups[group_of(m, t)];
+    r.a0 = g.a0;
+    r.a1 = g.a1;
+    r.b0 = g.b0;
+    r.b1 = g.b1;
+    return r;
+  }
   if (m.mode == kModeBlockCausal) {
     r.a1 = (t / m.c + 1) * m.c;
     r.b0 = r.b1 = 0;
@@ -61,10 +96,13 @@ AJVP_HD RowRange row_range(const MaskSpec& m, int t) {
   return r;
 }
 
-AJVP_HD bool row_allows(const RowRange& r, int k) { return k < r.a1 || (k >= r.b0 && k < r.b1); }
+AJVP_HD bool row_allows(const RowRange& r, int k) {
+  return (k >= r.a0 && k < r.a1) || (k >= r.b0 && k < r.b1);
+}
 
 // First row after t whose admissible set may differ from row t's.
 AJVP_HD int next_group_start(const MaskSpec& m, int t) {
+  if (m.mode == kModeGroups) return m.groups[group_of(m, t)].row_end;
   if (m.mode == kModeTeacherForcing) {
     const int nc = m.n * m.c;
     if (t >= nc) return nc + ((t - nc) / m.c + 1) * m.c;
@@ -72,21 +110,24 @@ AJVP_HD int next_group_start(const MaskSpec& m, int t) {
   return (t / m.c + 1) * m.c;
 }
 
-// Key-tile schedule of one query tile: the tiles [0, n1) and then
+// Key-tile schedule of one query tile: the tiles [t1_begin, t1_end) and then
 // [t2_begin, t2_end); a tile is "full" when every pair in it is admissible
 // for every valid row of the query tile.
 struct TileSched {
-  int n1;
+  int t1_begin, t1_end;
   int t2_begin, t2_end;
-  int i_a1;        // intersection, first part [0, i_a1)
+  int i_a0, i_a1;  // intersection, first part [i_a0, i_a1) (may be empty)
   int i_b0, i_b1;  // intersection, second part [i_b0, i_b1) (may be empty)
   int bn;
 
-  AJVP_HD int count() const { return n1 + (t2_end - t2_begin); }
-  AJVP_HD int tile(int idx) const { return idx < n1 ? idx : t2_begin + (idx - n1); }
+  AJVP_HD int count() const { return (t1_end - t1_begin) + (t2_end - t2_begin); }
+  AJVP_HD int tile(int idx) const {
+    const int n1 = t1_end - t1_begin;
+    return idx < n1 ? t1_begin + idx : t2_begin + (idx - n1);
+  }
   AJVP_HD bool full(int kt) const {
     const int k0 = kt * bn, k1 = k0 + bn;
-    return k1 <= i_a1 || (k0 >= i_b0 && k1 <= i_b1);
+    return (k0 >= i_a0 && k1 <= i_a1) || (k0 >= i_b0 && k1 <= i_b1);
   }
 };
 
@@ -96,12 +137,17 @@ AJVP_HD int cdiv(int a, int b) { return (a + b - 1) / b; }
 AJVP_HD TileSched make_tile_sched(const MaskSpec& m, int q_tile, int bm, int bn) {
   const int r0 = q_tile * bm;
   const int r1 = (r0 + bm < m.L) ? r0 + bm : m.L;
-  int u_a1 = 0, u_b0 = 0x7fffffff, u_b1 = 0;  // union
-  int x_a1 = 0x7fffffff, x_b0 = 0, x_b1 = 0;  // intersection
+  int u_a0 = 0x7fffffff, u_a1 = 0, u_b0 = 0x7fffffff, u_b1 = 0;  // union (non-empty parts)
+  int x_a0 = 0, x_a1 = 0x7fffffff;                                 // intersection, first part
+  int x_b0 = 0, x_b1 = 0;
   bool all_b = true, b_set = false, b_same = true;
   for (int t = r0; t < r1;) {
     const RowRange r = row_range(m, t);
-    if (r.a1 > u_a1) u_a1 = r.a1;
+    if (r.a1 > r.a0) {
+      if (r.a0 < u_a0) u_a0 = r.a0;
+      if (r.a1 > u_a1) u_a1 = r.a1;
+    }
+    if (r.a0 > x_a0) x_a0 = r.a0;
     if (r.a1 < x_a1) x_a1 = r.a1;
     if (r.b1 > r.b0) {
       if (r.b0 < u_b0) u_b0 = r.b0;
@@ -110,7 +156,7 @@ AJVP_HD TileSched make_tile_sched(const MaskSpec& m, int q_tile, int bm, int bn)
         x_b0 = r.b0;
         x_b1 = r.b1;
         b_set = true;
-      } else if (r.b0 != x_b0) {
+      } else if (r.b0 != x_b0 || r.b1 != x_b1) {
         b_same = false;
       }
     } else {
@@ -118,30 +164,41 @@ AJVP_HD TileSched make_tile_sched(const MaskSpec& m, int q_tile, int bm, int bn)
     }
     t = next_group_start(m, t);
   }
-  const bool any_b = b_set;
   TileSched s;
   s.bn = bn;
-  s.i_a1 = (x_a1 == 0x7fffffff) ? 0 : x_a1;
+  s.i_a0 = x_a0;
+  s.i_a1 = (x_a1 == 0x7fffffff || x_a1 < x_a0) ? x_a0 : x_a1;
   if (all_b && b_set && b_same) {
     s.i_b0 = x_b0;
     s.i_b1 = x_b1;
   } else {
     s.i_b0 = s.i_b1 = 0;
   }
+  const bool any_a = u_a1 > 0 && u_a0 != 0x7fffffff;
+  const bool any_b = b_set;
+  s.t1_begin = s.t1_end = s.t2_begin = s.t2_end = 0;
+  if (!any_a && !any_b) return s;
   if (!any_b) {
-    s.n1 = cdiv(u_a1, bn);
-    s.t2_begin = s.t2_end = 0;
+    s.t1_begin = u_a0 / bn;
+    s.t1_end = cdiv(u_a1, bn);
     return s;
   }
+  if (!any_a) {
+    s.t1_begin = u_b0 / bn;
+    s.t1_end = cdiv(u_b1, bn);
+    return s;
+  }
+  const int lo = u_a0 < u_b0 ? u_a0 : u_b0;
   if (u_b0 <= u_a1) {  // the two parts touch: one contiguous range
     const int hi = u_b1 > u_a1 ? u_b1 : u_a1;
-    s.n1 = cdiv(hi, bn);
-    s.t2_begin = s.t2_end = 0;
+    s.t1_begin = lo / bn;
+    s.t1_end = cdiv(hi, bn);
     return s;
   }
-  s.n1 = cdiv(u_a1, bn);
+  s.t1_begin = u_a0 / bn;
+  s.t1_end = cdiv(u_a1, bn);
   int b_begin = u_b0 / bn;
-  if (b_begin < s.n1) b_begin = s.n1;  // a tile shared by both parts is listed once
+  if (b_begin < s.t1_end) b_begin = s.t1_end;  // a tile shared by both parts is listed once
   s.t2_begin = b_begin;
   s.t2_end = cdiv(u_b1, bn);
   if (s.t2_end < s.t2_begin) s.t2_end = s.t2_begin;

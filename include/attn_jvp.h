@@ -81,6 +81,23 @@ typedef struct {
   int32_t n_chunks;     /* n >= 1 */
 } attn_jvp_mask;
 
+/*
+ * General masks (Causal-rCM summary page, App. B: the kernel takes masks as
+ * query groups with admissible key ranges). Group g covers the query rows
+ * [row_end of group g-1 (0 for g = 0), row_end of group g); each of those rows
+ * may attend to keys [k0_begin, k0_end) and [k1_begin, k1_end). A table lists
+ * 1 to ATTN_JVP_MAX_GROUPS groups in row order, the last ending at L, with
+ * 0 <= k0_begin <= k0_end <= k1_begin <= k1_end <= L and at least one key per
+ * group (either range may be empty). The teacher-forcing mask is such a table
+ * with one group per chunk of rows (clean chunks, then noisy chunks).
+ */
+#define ATTN_JVP_MAX_GROUPS 512
+typedef struct {
+  int32_t row_end;
+  int32_t k0_begin, k0_end;
+  int32_t k1_begin, k1_end;
+} attn_jvp_group;
+
 /* ---- problem --------------------------------------------------------- */
 typedef enum {
   ATTN_JVP_BF16 = 0, /* bf16 inputs/outputs, fp32 accumulation, tensor cores */
@@ -118,6 +135,30 @@ int attn_jvp_fwd(const attn_jvp_shape* shape,
                  attn_jvp_mask mask,
                  void* o, void* to, float* lse,
                  void* stream);
+
+/*
+ * attn_jvp_fwd_groups - attn_jvp_fwd with a general mask given as a table of
+ * row groups (see attn_jvp_group) instead of {mode, c, n}: same operation,
+ * layouts, outputs and asynchronous behaviour.
+ *
+ *   groups    host array of n_groups groups; read during the call only (it is
+ *             copied into the launch), the caller keeps ownership
+ *   n_groups  1 .. ATTN_JVP_MAX_GROUPS
+ *
+ * Returns ATTN_JVP_ERR_INVALID_ARGUMENT for a table that breaks the rules
+ * above (rows not increasing to L, ranges out of order or outside [0, L), a
+ * group with no key) and ATTN_JVP_ERR_UNSUPPORTED for more than
+ * ATTN_JVP_MAX_GROUPS groups; nothing is launched then. Each query block is
+ * scheduled over the union of its rows' ranges, so key tiles in a gap of that
+ * union are visited (and fully masked); tables whose neighbouring groups have
+ * similar ranges waste little.
+ */
+int attn_jvp_fwd_groups(const attn_jvp_shape* shape,
+                        const void* q, const void* k, const void* v,
+                        const void* tq, const void* tk, const void* tv,
+                        const attn_jvp_group* groups, int32_t n_groups,
+                        void* o, void* to, float* lse,
+                        void* stream);
 
 /*
  * attn_jvp_fwd_host - the same operation on HOST buffers: copies the six
@@ -218,6 +259,15 @@ int64_t attn_jvp_unmasked_pairs(attn_jvp_mask mask);
 int32_t attn_jvp_schedule_tiles(attn_jvp_mask mask, int64_t L, int32_t block_m,
                                 int32_t block_n, int32_t q_tile,
                                 int32_t* tiles, uint8_t* full, int32_t cap);
+
+/*
+ * attn_jvp_schedule_tiles_groups - the same for a group-table mask (the table
+ * validated as for attn_jvp_fwd_groups, L = its last row_end). Returns the
+ * number of key tiles or -1 on a bad argument.
+ */
+int32_t attn_jvp_schedule_tiles_groups(const attn_jvp_group* groups, int32_t n_groups, int64_t L,
+                                       int32_t block_m, int32_t block_n, int32_t q_tile,
+                                       int32_t* tiles, uint8_t* full, int32_t cap);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
 int32_t attn_jvp_version(void);

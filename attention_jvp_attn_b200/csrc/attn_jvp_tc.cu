@@ -589,14 +589,21 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
     // enough: a warpgroup writes its next tile's value only after that tile's
     // S is ready, and that S is issued only once every softmax warp has
     // arrived on s_free, which each does after reading this value. Bounded spin.
-    auto exchange_max = [&](float mine, float& theirs) -> bool {
+    // The swap is split: publish this warpgroup's maxima, compute P with the
+    // running max meanwhile, then read the other's (normally long there).
+    auto publish_max = [&](float mine) {
       *my_x = mine;
       __syncwarp();
       ++xseq;
-      int ok = 1;
       if (lane == 0) {
         __threadfence_block();
         *my_flag = xseq;
+      }
+      __syncwarp();
+    };
+    auto read_max = [&](float& theirs) -> bool {
+      int ok = 1;
+      if (lane == 0) {
         uint32_t polls = 0;
         uint64_t t0 = 0;
         while (static_cast<int>(*other_flag - xseq) < 0) {
@@ -683,10 +690,34 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
           mx3 = fmaxf(mx3, __uint_as_float(sr[j + 3]));
         }
         const float my_max = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        tc_fence_before();
+        publish_max(my_max);
+        // P of this half tile at the running max mb (bf16, packed) and its row sum.
+        uint32_t pk[C::HALF / 2];
+        float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
+        auto compute_p = [&](float mb) {
+          ls0 = ls1 = ls2 = ls3 = 0.f;
+#pragma unroll
+          for (int j = 0; j < C::HALF / 2; j += 2) {
+            const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * j]), scale_log2, -mb));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * j + 1]), scale_log2, -mb));
+            const float p2 = ex2_approx(fmaf(__uint_as_float(sr[2 * j + 2]), scale_log2, -mb));
+            const float p3 = ex2_approx(fmaf(__uint_as_float(sr[2 * j + 3]), scale_log2, -mb));
+            ls0 += p0;
+            ls1 += p1;
+            ls2 += p2;
+            ls3 += p3;
+            pk[j] = pack_bf16x2(p0, p1);
+            pk[j + 1] = pack_bf16x2(p2, p3);
+          }
+        };
+        // Speculate that the running max stays (it does unless a row's max grows
+        // by more than kRescaleTau): P first, the other half's maxima after.
+        const bool spec = __all_sync(0xffffffffu, m_use != -INFINITY);
+        if (spec) compute_p(m_use);
         // row maximum over both halves of the tile
         float their_max;
-        tc_fence_before();
-        if (!exchange_max(my_max, their_max)) { ok = false; break; }
+        if (!read_max(their_max)) { ok = false; break; }
         // S_g is in registers and both warpgroups have read this tile's maxima:
         // the MMA warp may write S_{g+1} over S_g.
         __syncwarp();
@@ -706,6 +737,9 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
           dsum *= alpha;
           resc = true;
         }
+        // (re)compute P when it was not speculated or the running max moved
+        if (!spec || __any_sync(0xffffffffu, resc)) compute_p((m_use == -INFINITY) ? 0.f : m_use);
+        // A and T to the new running max (S is no longer needed here)
         if (__any_sync(0xffffffffu, resc)) {
           // Every value MMA of earlier tiles has completed once this tile's
           // tS' has (it is issued after them and they run in issue order).
@@ -729,22 +763,6 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
             for (int j = 0; j < 32; ++j) a[j] = __float_as_uint(__uint_as_float(a[j]) * alpha);
             tmem_st32(tT + 32 * c, a);
           }
-        }
-        const float mb = (m_use == -INFINITY) ? 0.f : m_use;
-        uint32_t pk[C::HALF / 2];
-        float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
-#pragma unroll
-        for (int j = 0; j < C::HALF / 2; j += 2) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * j]), scale_log2, -mb));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * j + 1]), scale_log2, -mb));
-          const float p2 = ex2_approx(fmaf(__uint_as_float(sr[2 * j + 2]), scale_log2, -mb));
-          const float p3 = ex2_approx(fmaf(__uint_as_float(sr[2 * j + 3]), scale_log2, -mb));
-          ls0 += p0;
-          ls1 += p1;
-          ls2 += p2;
-          ls3 += p3;
-          pk[j] = pack_bf16x2(p0, p1);
-          pk[j + 1] = pack_bf16x2(p2, p3);
         }
         l += (ls0 + ls1) + (ls2 + ls3);
         if (warp == 0 && lane == 0) AJVP_EV(g, 7);

@@ -7,8 +7,11 @@
 #include <cmath>
 #include <cstddef>
 #include <cstring>
+#include <functional>
 #include <mutex>
 #include <numeric>
+#include <queue>
+#include <utility>
 #include <vector>
 
 #include "attn_jvp.h"
@@ -225,6 +228,40 @@ int fill_order(const MaskSpec& ms, int n_qtiles, int bm, uint16_t* order) {
   return n_qtiles;
 }
 
+// Work lists for `units` units of the persistent grid: head by head (so that
+// running units share a head's keys in L2), each query block of the head goes,
+// longest first, to the unit with the least work so far (ties: lowest unit).
+// Work is the block's key-tile count. Returns false if the lists do not fit.
+bool fill_work_lists(const MaskSpec& ms, int bh_count, int n_qtiles, int bm, int units,
+                     const uint16_t* head_order, uint16_t* lists, uint16_t* unit_start) {
+  const int n_items = bh_count * n_qtiles;
+  if (n_items > ajvp::kMaxOrder || units < 1 || units > ajvp::kMaxUnits) return false;
+  std::vector<int> cost(n_qtiles);
+  for (int t = 0; t < n_qtiles; ++t)
+    cost[t] = ajvp::make_tile_sched(ms, t, bm, ajvp::kTcBlockN).count();
+  using Load = std::pair<int64_t, int>;  // (work so far, unit)
+  std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+  for (int u = 0; u < units; ++u) heap.push({0, u});
+  std::vector<std::vector<uint16_t>> per(units);
+  for (int bh = 0; bh < bh_count; ++bh) {
+    for (int r = 0; r < n_qtiles; ++r) {
+      const int qt = head_order ? head_order[r] : n_qtiles - 1 - r;
+      Load x = heap.top();
+      heap.pop();
+      per[x.second].push_back(static_cast<uint16_t>(bh * n_qtiles + qt));
+      x.first += cost[qt];
+      heap.push(x);
+    }
+  }
+  int at = 0;
+  for (int u = 0; u < units; ++u) {
+    unit_start[u] = static_cast<uint16_t>(at);
+    for (uint16_t pos : per[u]) lists[at++] = pos;
+  }
+  unit_start[units] = static_cast<uint16_t>(at);
+  return true;
+}
+
 int launch_bf16(DeviceState* st, const attn_jvp_shape* s, const void* q, const void* k,
                 const void* v, const void* tq, const void* tk, const void* tv, const MaskSpec& ms,
                 void* o, void* to, float* lse, cudaStream_t stream) {
@@ -261,6 +298,16 @@ int launch_bf16(DeviceState* st, const attn_jvp_shape* s, const void* q, const v
 #endif
   const int grid = pair ? 2 * std::min(st->pair_clusters, p.n_items)
                         : std::min(st->sm_count, p.n_items);
+  {
+    static thread_local uint16_t head_order[ajvp::kMaxOrder];
+    const bool have_order = p.order_len > 0;
+    if (have_order) std::memcpy(head_order, p.order, sizeof(uint16_t) * p.n_qtiles);
+    p.list_mode = fill_work_lists(ms, p.B * p.H, p.n_qtiles, bmu, pair ? grid / 2 : grid,
+                                  have_order ? head_order : nullptr, p.order, p.unit_start)
+                      ? 1
+                      : 0;
+    if (!p.list_mode && have_order) std::memcpy(p.order, head_order, sizeof(uint16_t) * p.n_qtiles);
+  }
   if (ajvp::tc_launch(static_cast<int>(s->d), p, grid, stream) != cudaSuccess)
     return ATTN_JVP_ERR_CUDA;
   return ATTN_JVP_OK;

@@ -6,8 +6,8 @@
 // tangent; the same sparse (query tile x key range) schedule drives the primal
 // and tangent scores; queries and keys are tiled; outputs are O, LSE and tO.
 //
-// Per query tile (128 rows, one TMEM lane per row) and admissible key tile j
-// (128 keys), with s the softmax scale and x = s log2(e) Q K^T:
+// Per query tile (128 rows per CTA, one TMEM lane per row) and admissible key
+// tile j (128 keys), with s the softmax scale and x = s log2(e) Q K^T:
 //   MMA   S_j   = Q K_j^T                      (TMEM cols [0,128),   fp32)
 //   MMA   tS'_j = tQ K_j^T + Q tK_j^T          (TMEM cols [128,256), fp32)
 //   warps p = 2^(x - m), l += sum p;  u = p * s * tS', D += sum u;
@@ -24,15 +24,21 @@
 // m_new)) when a tile's max exceeds it by more than kRescaleTau: every p stays
 // <= 2^kRescaleTau and the final normalisation by l is exact.
 //
-// Warp roles (320 threads, one CTA per SM, persistent over work items):
+// Head dim 128 runs on CTA pairs (clusters of two SMs, cta_group::2 MMAs over
+// 256 query rows, each SM holding half of every key/value tile); head dim 64
+// on single CTAs. Warp roles (320 threads, one CTA per SM, persistent):
 //   warps 0-7  softmax + epilogue: two warpgroups, each owning half of the
 //              key columns of a tile (and half of the output columns)
-//   warp  8    TMA producer (one thread): Q,tQ per item; K,tK,tV,V per key tile
-//   warp  9    MMA issuer (one thread), TMEM allocator
-// Work items (batch, head, query tile) are ordered head-major so that CTAs
-// running at the same time share one head's keys in L2, and, within a head,
-// longest first; CTA c takes items c, 2G-1-c, 2G+c, ... of that list.
-// No TMA multicast is used anywhere: each CTA loads its own tiles.
+//   warp  8    TMA producer (warp-wide, one elected lane issues): Q,tQ per
+//              item; (K,tK) and (tV,V) ring elements per key tile
+//   warp  9    MMA issuer (warp-wide, elect.sync; the pair's leader only),
+//              TMEM allocator
+// Work items (batch, head, query row block) are handed out head by head so
+// that units running at the same time share one head's keys in L2: from host
+// work lists (each block, longest first, to the unit with the least work), or
+// in snake rounds over a longest-first order when the lists do not fit.
+// No TMA multicast is used anywhere: each CTA loads its own tiles (a pair's
+// copies complete on the leader's barriers, the cta_group::2 form).
 #include <cuda_bf16.h>
 
 #include "kernels.cuh"
@@ -183,8 +189,15 @@ __device__ __forceinline__ int item_position(int k, int cta, int G) {
   return (k & 1) ? k * G + (G - 1 - cta) : k * G + cta;
 }
 
-// First work item of this CTA at round >= k (k is advanced to it).
+// The unit's k-th work item (work lists), or its first item at snake round
+// >= k (k is advanced to it).
 __device__ __forceinline__ bool next_item(const TcParams& p, int cta, int G, int& k, int& pos) {
+  if (p.list_mode) {
+    const int i = p.unit_start[cta] + k;
+    if (i >= p.unit_start[cta + 1]) return false;
+    pos = p.order[i];
+    return true;
+  }
   for (; k * G < p.n_items; ++k) {
     pos = item_position(k, cta, G);
     if (pos < p.n_items) return true;
@@ -196,7 +209,7 @@ __device__ __forceinline__ WorkItem decode_item(const TcParams& p, int pos) {
   const int bh = pos / p.n_qtiles;
   const int r = pos - bh * p.n_qtiles;
   WorkItem w;
-  w.qt = p.order_len ? static_cast<int>(p.order[r]) : (p.n_qtiles - 1 - r);
+  w.qt = p.list_mode ? r : (p.order_len ? static_cast<int>(p.order[r]) : (p.n_qtiles - 1 - r));
   w.b = bh / p.H;
   w.h = bh - w.b * p.H;
   return w;

@@ -13,7 +13,8 @@ namespace ajvp {
 constexpr int kTcBlockM = 128;   // query rows per tile (one TMEM lane per row)
 constexpr int kTcBlockN = 128;   // keys per tile
 constexpr int kTcThreads = 320;  // warps 0-7 softmax+epilogue, 8 TMA producer, 9 MMA issuer
-constexpr int kMaxOrder = 4096;  // longest-first query-tile order table capacity
+constexpr int kMaxOrder = 4096;  // order table / work-list capacity
+constexpr int kMaxUnits = 160;   // work lists: units (CTAs or CTA pairs) of the persistent grid
 
 struct TcParams {
   CUtensorMap map_q, map_k, map_v, map_tq, map_tk, map_tv;  // [B, L, H, d] bf16, 128B swizzle
@@ -27,7 +28,12 @@ struct TcParams {
   MaskSpec mask;
   float scale_log2;  // s * log2(e)
   float scale;       // s
-  int order_len;     // n_qtiles if `order` is filled, else 0 (reverse index order)
+  int order_len;     // n_qtiles if `order` is a per-head order table, else 0 (reverse index order)
+  // list_mode: unit u runs the items order[unit_start[u] .. unit_start[u+1]), each an item
+  // position b*H*n_qtiles + h*n_qtiles + qt; else unit u takes rounds of a snake over
+  // positions, with the query block of position r within a head given by the order table
+  int list_mode;
+  uint16_t unit_start[kMaxUnits + 1];
 #ifdef AJVP_TRACE
   long long* trace;  // per-tile event clocks of one CTA (trace builds only)
 #endif

@@ -390,6 +390,57 @@ def run_gpu(args):
     return 0
 
 
+def run_sweep(args) -> int:
+    """Sweep (config 5): every point of inputs.sweep_points() on one GPU, one
+    JSON line each (CUDA-event median of `--steps` launches after `--warmup`),
+    then a summary line. Device timing only; inputs resident."""
+    import torch
+    import attention_jvp_attn_b200 as aj
+    from attention_jvp_attn_b200 import inputs as wl
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        raise SystemExit("--sweep runs on one GPU")
+    dev = torch.device("cuda", 0)
+    peaks, _ = load_peaks()
+    peak = peaks["bf16_tflops"]
+    rows = []
+    for w in wl.sweep_points():
+        x = wl.make_inputs(w, device=dev)
+        o = torch.empty_like(x["q"])
+        to = torch.empty_like(x["q"])
+        lse = torch.empty((w.B, w.H, w.L), dtype=torch.float32, device=dev)
+
+        def step():
+            aj.attn_jvp(x["q"], x["k"], x["v"], x["tq"], x["tk"], x["tv"], w.mode,
+                        w.chunk_tokens, w.n_chunks, w.scale, out=(o, to, lse))
+
+        for _ in range(max(args.warmup, 1)):
+            step()
+        if aj.sync_status(dev) != 0:
+            raise SystemExit(f"device status error on {w.name}")
+        ms = []
+        for _ in range(args.steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            step()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            ms.append(e0.elapsed_time(e1))
+        ms.sort()
+        med = ms[len(ms) // 2]
+        tf = flops_per_step(w) / (med * 1e-3) / 1e12
+        row = {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d,
+               "chunk_tokens": w.chunk_tokens, "n_chunks": w.n_chunks, "ms": med,
+               "tflops": tf, "pct_of_peak": 100.0 * tf / peak}
+        rows.append(row)
+        print(json.dumps(row), flush=True)
+        del x, o, to, lse
+        torch.cuda.empty_cache()
+    tfs = sorted(r["tflops"] for r in rows)
+    print(json.dumps({"sweep_points": len(rows), "tflops_min": tfs[0], "tflops_median": tfs[len(tfs) // 2],
+                      "tflops_max": tfs[-1], "unit": "TFLOP/s", "peak": peak}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -403,11 +454,15 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--ref-budget", type=float, default=6.0)
+    ap.add_argument("--sweep", action="store_true",
+                    help="time every sweep point (config 5) on one GPU, one JSON line each")
     args = ap.parse_args()
     if args.warmup < 0 or args.steps < 1:
         raise SystemExit("need --steps >= 1 and --warmup >= 0")
     if args.impl == "reference":
         return run_reference(args)
+    if args.sweep:
+        return run_sweep(args)
     return run_gpu(args)
 
 

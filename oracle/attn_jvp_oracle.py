@@ -40,6 +40,11 @@ share an admissible key set made of at most two key ranges. The groups cover
 the rows [0, L) in order; group g holds rows [row_end of g-1, row_end of g)
 (0 for the first) and admits keys [k0_begin, k0_end) and [k1_begin, k1_end).
 
+Backward (for training the student; the pages return LSE so that a backward
+pass can rebuild P): attn_vjp_rows / attn_vjp_dense give dQ, dK, dV from an
+output cotangent dO and an optional LSE cotangent, pinned separately by
+tests/test_oracle_vjp_pins.py.
+
 Every function here is pinned by tests/test_oracle_pins.py against values
 that do not come from this file: finite differences, an autodiff JVP of the
 library softmax attention, hand-derived closed forms, hand-written masks,
@@ -219,6 +224,61 @@ def attn_forward_dense(q, k, v, mode: int, c: int, n: int,
     z = np.zeros_like(_as64(q))
     O, _, lse = attn_jvp_dense(q, k, v, z, z, z, mode, c, n, scale)
     return O, lse
+
+
+def attn_vjp_rows(q, k, v, do, mode: int, c: int, n: int, scale: Optional[float],
+                  dlse=None, groups: Optional[Sequence[Group]] = None
+                  ) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Backward (vector-Jacobian product) of the masked primal attention of ONE
+    (batch, head): given the output cotangent dO [L, d] (and optionally a
+    cotangent dLSE [L] of the log-sum-exp), returns dQ, dK, dV [L, d].
+
+    This is the gradient the primal network needs during training; the pages
+    return LSE with the forward so a backward pass can rebuild P from it
+    (Causal-rCM summary page, App. B, last item). Plain definition, with P the
+    masked softmax of S = s q k^T:
+        dV = P^T dO
+        dP = dO V^T
+        Delta_i = sum_j P_ij dP_ij   (= dO_i . O_i)
+        dS = P * (dP - Delta) + P * dLSE_i
+        dQ = s dS K,   dK = s dS^T Q
+    (d LSE_i / d S_ij = P_ij gives the last term of dS.)"""
+    q, k, v, do = (_as64(x) for x in (q, k, v, do))
+    L, d = q.shape
+    s = (1.0 / math.sqrt(d)) if scale is None else float(scale)
+    t = np.arange(L)
+    if groups is not None:
+        M = allowed_groups(groups, t[:, None], t[None, :])
+    else:
+        M = allowed(mode, c, n, t[:, None], t[None, :])
+    S = np.where(M, s * (q @ k.T), -np.inf)
+    smax = S.max(axis=1, keepdims=True)
+    lse = smax[:, 0] + np.log(np.exp(S - smax).sum(axis=1))
+    P = np.exp(S - lse[:, None])
+    dV = P.T @ do
+    dP = do @ v.T
+    delta = (P * dP).sum(axis=1, keepdims=True)
+    dS = P * (dP - delta)
+    if dlse is not None:
+        dS = dS + P * _as64(dlse)[:, None]
+    dQ = s * (dS @ k)
+    dK = s * (dS.T @ q)
+    return dQ, dK, dV
+
+
+def attn_vjp_dense(q, k, v, do, mode: int, c: int, n: int, scale: Optional[float] = None,
+                   dlse=None, groups: Optional[Sequence[Group]] = None):
+    """dQ, dK, dV [B, L, H, d] for [B, L, H, d] inputs and output cotangent dO
+    (dLSE [B, H, L] optional), all float64 numpy."""
+    q, k, v, do = (_as64(x) for x in (q, k, v, do))
+    B, L, H, d = q.shape
+    dQ, dK, dV = (np.empty((B, L, H, d)) for _ in range(3))
+    for b in range(B):
+        for h in range(H):
+            g = attn_vjp_rows(q[b, :, h], k[b, :, h], v[b, :, h], do[b, :, h], mode, c, n, scale,
+                              None if dlse is None else _as64(dlse)[b, h], groups)
+            dQ[b, :, h], dK[b, :, h], dV[b, :, h] = g
+    return dQ, dK, dV
 
 
 def effective_flops(pairs: int, d: int) -> int:

@@ -20,7 +20,7 @@ from . import _abi
 from ._abi import AttnJvpError  # noqa: F401
 from .inputs import BLOCK_CAUSAL, TEACHER_FORCING  # noqa: F401
 
-__all__ = ["attn_jvp", "attn_jvp_groups", "attn_jvp_host", "sync_status", "unmasked_pairs", "schedule_tiles",
+__all__ = ["attn_jvp", "attn_jvp_groups", "attn_jvp_bwd", "attn_jvp_bwd_groups", "attn_jvp_host", "sync_status", "unmasked_pairs", "schedule_tiles",
            "host_staging_bytes", "AttnJvpError", "TEACHER_FORCING", "BLOCK_CAUSAL"]
 
 _DT = {torch.bfloat16: _abi.DTYPE_BF16, torch.float32: _abi.DTYPE_F32}
@@ -107,6 +107,61 @@ def attn_jvp_groups(q, k, v, tq, tk, tv, groups: Sequence[Tuple[int, int, int, i
                                      lse.data_ptr(), _stream_handle(q.device))
     _abi.check(rc, "attn_jvp_fwd_groups")
     return o, to, lse
+
+
+def _bwd_args(q, k, v, o, do, lse, dlse, scale, out):
+    for t in (q, k, v, o, do):
+        if not t.is_cuda:
+            raise ValueError("inputs must be CUDA tensors")
+        if t.shape != q.shape or t.dtype != q.dtype or t.device != q.device:
+            raise ValueError("q, k, v, o, do must share shape, dtype and device")
+        if not t.is_contiguous():
+            raise ValueError("inputs must be contiguous [B, L, H, d]")
+    B, L, H, d = q.shape
+    for t in (lse,) + ((dlse,) if dlse is not None else ()):
+        if t.shape != (B, H, L) or t.dtype != torch.float32 or t.device != q.device \
+                or not t.is_contiguous():
+            raise ValueError("lse and dlse must be contiguous fp32 [B, H, L] on the inputs' device")
+    shape = _shape(q, scale)
+    if out is None:
+        out = (torch.empty_like(q), torch.empty_like(q), torch.empty_like(q))
+    return shape, out
+
+
+def attn_jvp_bwd(q, k, v, o, do, lse, mode: int, chunk_tokens: int, n_chunks: int,
+                 scale: Optional[float] = None, dlse: Optional[torch.Tensor] = None,
+                 out: Optional[Tuple[torch.Tensor, torch.Tensor, torch.Tensor]] = None):
+    """dQ, dK, dV ([B, L, H, d], input dtype) of the masked primal attention,
+    from the forward's inputs, its output O and LSE, the cotangent dO of O and
+    optionally a cotangent dLSE of LSE ([B, H, L] fp32), on the current stream."""
+    shape, (dq, dk, dv) = _bwd_args(q, k, v, o, do, lse, dlse, scale, out)
+    lib = _abi.load()
+    with torch.cuda.device(q.device):
+        rc = lib.attn_jvp_bwd(ctypes.byref(shape), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                              o.data_ptr(), do.data_ptr(), lse.data_ptr(),
+                              dlse.data_ptr() if dlse is not None else None,
+                              _mask(mode, chunk_tokens, n_chunks),
+                              dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                              _stream_handle(q.device))
+    _abi.check(rc, "attn_jvp_bwd")
+    return dq, dk, dv
+
+
+def attn_jvp_bwd_groups(q, k, v, o, do, lse, groups: Sequence[Tuple[int, int, int, int, int]],
+                        scale: Optional[float] = None, dlse: Optional[torch.Tensor] = None,
+                        out: Optional[Tuple[torch.Tensor, torch.Tensor, torch.Tensor]] = None):
+    """attn_jvp_bwd with a group-table mask (as for attn_jvp_groups)."""
+    shape, (dq, dk, dv) = _bwd_args(q, k, v, o, do, lse, dlse, scale, out)
+    table = _abi.group_array(groups)
+    lib = _abi.load()
+    with torch.cuda.device(q.device):
+        rc = lib.attn_jvp_bwd_groups(ctypes.byref(shape), q.data_ptr(), k.data_ptr(),
+                                     v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
+                                     dlse.data_ptr() if dlse is not None else None,
+                                     table, len(groups), dq.data_ptr(), dk.data_ptr(),
+                                     dv.data_ptr(), _stream_handle(q.device))
+    _abi.check(rc, "attn_jvp_bwd_groups")
+    return dq, dk, dv
 
 
 def host_staging_bytes(B: int, L: int, H: int, d: int, dtype: torch.dtype) -> int:

@@ -96,6 +96,13 @@ def load(path: str = None) -> ctypes.CDLL:
             ctypes.c_int32, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_uint8),
             ctypes.c_int32]
         lib.attn_jvp_schedule_tiles_groups.restype = ctypes.c_int32
+        lib.attn_jvp_bwd.argtypes = [ctypes.POINTER(Shape), vp, vp, vp, vp, vp, vp, vp, Mask,
+                                     vp, vp, vp, vp]
+        lib.attn_jvp_bwd.restype = ctypes.c_int
+        lib.attn_jvp_bwd_groups.argtypes = [ctypes.POINTER(Shape), vp, vp, vp, vp, vp, vp, vp,
+                                            ctypes.POINTER(Group), ctypes.c_int32, vp, vp, vp,
+                                            vp]
+        lib.attn_jvp_bwd_groups.restype = ctypes.c_int
         lib.attn_jvp_version.argtypes = []
         lib.attn_jvp_version.restype = ctypes.c_int32
         _lib = lib

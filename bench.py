@@ -73,8 +73,12 @@ def load_peaks():
 
 
 def kernel_source_hash() -> str:
+    """Hash of the sources the forward kernels are built from (the backward's
+    own source file does not change them)."""
     h = hashlib.sha256()
     for p in sorted(glob.glob(os.path.join(ROOT, "attention_jvp_attn_b200", "csrc", "*"))):
+        if os.path.basename(p).startswith("attn_jvp_bwd"):
+            continue
         with open(p, "rb") as f:
             h.update(os.path.basename(p).encode())
             h.update(f.read())
@@ -441,6 +445,67 @@ def run_sweep(args) -> int:
     return 0
 
 
+def run_backward(args) -> int:
+    """Backward of the primal attention (attn_jvp_bwd) on one GPU: dQ, dK, dV
+    from the workload's Q, K, V, the forward's O and LSE and a seeded random
+    cotangent dO. One JSON line: CUDA-event median over `--steps` calls after
+    `--warmup`, inputs resident. Effective FLOPs count 10 d per admissible
+    pair (the products S, dP, dV, dK, dQ at 2 d each); the fp32 CUDA-core
+    kernels execute 7 d fused multiply-adds per pair (14 d FLOPs), against a
+    peak of 148 SMs x 128 fp32 lanes x 2 FLOPs x the sampled SM clock."""
+    import torch
+    import attention_jvp_attn_b200 as aj
+    from attention_jvp_attn_b200 import inputs as wl
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        raise SystemExit("--backward runs on one GPU")
+    dev = torch.device("cuda", 0)
+    w = workload_by_name(args.workload, args.heads)
+    x = wl.make_inputs(w, device=dev)
+    o, _, lse = aj.attn_jvp(x["q"], x["k"], x["v"], x["tq"], x["tk"], x["tv"], w.mode,
+                            w.chunk_tokens, w.n_chunks, w.scale)
+    del x["tq"], x["tk"], x["tv"]
+    g = torch.Generator(device=dev).manual_seed(1234)
+    do = torch.randn(x["q"].shape, generator=g, device=dev).to(x["q"].dtype)
+    out = tuple(torch.empty_like(x["q"]) for _ in range(3))
+
+    def step():
+        aj.attn_jvp_bwd(x["q"], x["k"], x["v"], o, do, lse, w.mode, w.chunk_tokens, w.n_chunks,
+                        w.scale, out=out)
+
+    for _ in range(max(args.warmup, 1)):
+        step()
+    if aj.sync_status(dev) != 0:
+        raise SystemExit("device status error")
+    clocks = ClockSampler(0)
+    clocks.start()
+    ms = []
+    for _ in range(args.steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        step()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        ms.append(e0.elapsed_time(e1))
+    ck = clocks.stop()
+    ms.sort()
+    med = ms[len(ms) // 2]
+    pairs_total = flops_per_step(w) // (12 * w.d)
+    eff = 10 * w.d * pairs_total / (med * 1e-3) / 1e12
+    executed = 14 * w.d * pairs_total / (med * 1e-3) / 1e12
+    mhz = (ck or {}).get("sm_mhz") or 1965.0
+    alu_peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
+    print(json.dumps({"mode": "backward", "workload": w.name, "dtype": w.dtype,
+                      "B": w.B, "H": w.H, "L": w.L, "d": w.d, "steps": args.steps,
+                      "warmup": args.warmup, "ms": med, "ms_min": ms[0], "ms_max": ms[-1],
+                      "metric": "backward effective TFLOP/s (10 d per admissible pair)",
+                      "value": eff, "unit": "TFLOP/s",
+                      "roofline": {"bound": "alu", "achieved": executed, "peak": alu_peak,
+                                   "unit": "TFLOP/s", "frac": executed / alu_peak,
+                                   "note": "fp32 FMA pipe; 14 d FLOPs executed per pair"},
+                      "clocks": ck}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -456,6 +521,8 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=6.0)
     ap.add_argument("--sweep", action="store_true",
                     help="time every sweep point (config 5) on one GPU, one JSON line each")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward of the primal attention on one GPU (one JSON line)")
     args = ap.parse_args()
     if args.warmup < 0 or args.steps < 1:
         raise SystemExit("need --steps >= 1 and --warmup >= 0")
@@ -463,6 +530,8 @@ def main():
         return run_reference(args)
     if args.sweep:
         return run_sweep(args)
+    if args.backward:
+        return run_backward(args)
     return run_gpu(args)
 
 

@@ -233,6 +233,63 @@ int attn_jvp_fwd_noalloc(const attn_jvp_shape* shape,
                          void* o, void* to, float* lse,
                          void* stream);
 
+/* ---- backward of the primal attention --------------------------------- */
+
+/*
+ * attn_jvp_bwd - gradients dQ, dK, dV of the masked primal attention
+ * O = softmax(s Q K^T + M) V, for training the network whose forward
+ * attn_jvp_fwd computes. The fused forward returns LSE so that a backward
+ * pass can rebuild P without a second softmax pass (Causal-rCM summary page,
+ * App. B, last item); the pages say nothing more about the backward, and
+ * this is the plain gradient under the same mask:
+ *
+ *     P_ij  = exp(s q_i . k_j - LSE_i) on admissible pairs, 0 elsewhere
+ *     D_i   = dO_i . O_i - dLSE_i
+ *     dS_ij = P_ij ((dO_i . v_j) - D_i)
+ *     dV = P^T dO,    dK = s dS^T Q,    dQ = s dS K
+ *
+ * (dLSE is an optional cotangent of LSE; with it the result is the gradient
+ * of a loss that also depends on LSE.)
+ *
+ *   shape      as for attn_jvp_fwd (same dtype, d and scale rules)
+ *   q, k, v    device inputs of the forward, [B, L, H, d] of shape->dtype
+ *   o          the forward's output O, [B, L, H, d] of shape->dtype
+ *   dout       the cotangent dO of O, [B, L, H, d] of shape->dtype
+ *   lse        the forward's LSE, [B, H, L] float (natural log)
+ *   dlse       cotangent of LSE, [B, H, L] float, or NULL for none
+ *   mask       the forward's mask
+ *   dq, dk, dv device outputs, [B, L, H, d] of shape->dtype
+ *   stream     cudaStream_t to launch on
+ *
+ * All pointers 16-byte aligned; outputs must not overlap inputs or each
+ * other. Arithmetic is fp32 on CUDA cores for both dtypes; bf16 outputs are
+ * rounded to nearest even. Two launches (dQ per block of 32 query rows, dK
+ * and dV per block of 32 keys): each output element has one writer, so
+ * results are the same bits on every run. Keys that no row may attend to get
+ * zero gradients. lse must be the forward's (finite) LSE of these inputs.
+ *
+ * Returns ATTN_JVP_OK after enqueueing, or an error code with nothing
+ * launched (argument errors are found on the host before any device call).
+ * Does not synchronize; it has no bounded waits, so attn_jvp_sync_status
+ * reports only stream errors for it.
+ */
+int attn_jvp_bwd(const attn_jvp_shape* shape,
+                 const void* q, const void* k, const void* v,
+                 const void* o, const void* dout,
+                 const float* lse, const float* dlse,
+                 attn_jvp_mask mask,
+                 void* dq, void* dk, void* dv,
+                 void* stream);
+
+/* attn_jvp_bwd with a group-table mask (validated as for attn_jvp_fwd_groups). */
+int attn_jvp_bwd_groups(const attn_jvp_shape* shape,
+                        const void* q, const void* k, const void* v,
+                        const void* o, const void* dout,
+                        const float* lse, const float* dlse,
+                        const attn_jvp_group* groups, int32_t n_groups,
+                        void* dq, void* dk, void* dv,
+                        void* stream);
+
 /* ---- host-side helpers (need no GPU) ---------------------------------- */
 
 /* Number of admissible (query, key) pairs per (batch, head):

@@ -219,10 +219,11 @@ def attn_jvp_dense(q, k, v, tq, tk, tv, mode: int, c: int, n: int,
 
 
 def attn_forward_dense(q, k, v, mode: int, c: int, n: int,
-                       scale: Optional[float] = None):
-    """Primal output only (O and LSE); used to take finite differences."""
+                       scale: Optional[float] = None, groups: Optional[Sequence[Group]] = None):
+    """Primal output only (O and LSE); used to take finite differences and as
+    the forward whose O and LSE a backward pass starts from."""
     z = np.zeros_like(_as64(q))
-    O, _, lse = attn_jvp_dense(q, k, v, z, z, z, mode, c, n, scale)
+    O, _, lse = attn_jvp_dense(q, k, v, z, z, z, mode, c, n, scale, groups=groups)
     return O, lse
 
 

@@ -45,6 +45,10 @@ pass can rebuild P): attn_vjp_rows / attn_vjp_dense give dQ, dK, dV from an
 output cotangent dO and an optional LSE cotangent, pinned separately by
 tests/test_oracle_vjp_pins.py.
 
+Rotary position embedding of queries and keys (and their tangents) before
+the attention: rope_rotate / attn_jvp_rope_dense, pinned by
+tests/test_oracle_rope_pins.py.
+
 Every function here is pinned by tests/test_oracle_pins.py against values
 that do not come from this file: finite differences, an autodiff JVP of the
 library softmax attention, hand-derived closed forms, hand-written masks,
@@ -280,6 +284,44 @@ def attn_vjp_dense(q, k, v, do, mode: int, c: int, n: int, scale: Optional[float
                               None if dlse is None else _as64(dlse)[b, h], groups)
             dQ[b, :, h], dK[b, :, h], dV[b, :, h] = g
     return dQ, dK, dV
+
+
+def rope_rotate(x, cos, sin) -> np.ndarray:
+    """Rotary position embedding of x [B, L, H, d] with per-token angles given
+    as cos, sin [L, d/2]: each adjacent pair (x_2i, x_2i+1) of token t turns by
+    the angle phi_ti,
+        x'_2i   = x_2i cos phi_ti - x_2i+1 sin phi_ti
+        x'_2i+1 = x_2i sin phi_ti + x_2i+1 cos phi_ti.
+    The pages name RoPE as the positional treatment of Q and K and as a neighbour
+    of the attention inside the layer-level JVP (Causal-rCM summary page,
+    section 3, "KV Cache": pre- and post-RoPE caching); they give no formula, so
+    this is the standard rotary embedding on adjacent pairs, with the angles
+    (1-D or 3-D positions, the packed clean|noisy order) left to the caller."""
+    x = _as64(x)
+    c = _as64(cos)[None, :, None, :]
+    s = _as64(sin)[None, :, None, :]
+    a, b = x[..., 0::2], x[..., 1::2]
+    out = np.empty_like(x)
+    out[..., 0::2] = a * c - b * s
+    out[..., 1::2] = a * s + b * c
+    return out
+
+
+def attn_jvp_rope_dense(q, k, v, tq, tk, tv, cos, sin, mode: int, c: int, n: int,
+                        scale: Optional[float] = None, groups: Optional[Sequence[Group]] = None):
+    """O, tO, LSE of the attention JVP with RoPE applied to the queries and keys
+    first. The rotation does not depend on its input, so the tangents of the
+    rotated queries and keys are the rotated tangents."""
+    return attn_jvp_dense(rope_rotate(q, cos, sin), rope_rotate(k, cos, sin), v,
+                          rope_rotate(tq, cos, sin), rope_rotate(tk, cos, sin), tv,
+                          mode, c, n, scale, groups=groups)
+
+
+def rope_angles_1d(L: int, d: int, base: float = 10000.0) -> Tuple[np.ndarray, np.ndarray]:
+    """cos, sin [L, d/2] of 1-D positions 0..L-1 with frequencies base^(-2i/d)."""
+    t = np.arange(L, dtype=np.float64)[:, None]
+    theta = base ** (-2.0 * np.arange(d // 2, dtype=np.float64) / d)[None, :]
+    return np.cos(t * theta), np.sin(t * theta)
 
 
 def effective_flops(pairs: int, d: int) -> int:

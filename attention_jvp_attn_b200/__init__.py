@@ -20,7 +20,8 @@ from . import _abi
 from ._abi import AttnJvpError  # noqa: F401
 from .inputs import BLOCK_CAUSAL, TEACHER_FORCING  # noqa: F401
 
-__all__ = ["attn_jvp", "attn_jvp_groups", "attn_jvp_bwd", "attn_jvp_bwd_groups", "attn_jvp_host", "sync_status", "unmasked_pairs", "schedule_tiles",
+__all__ = ["attn_jvp", "attn_jvp_groups", "attn_jvp_bwd", "attn_jvp_bwd_groups", "rope",
+           "attn_jvp_rope", "attn_jvp_host", "sync_status", "unmasked_pairs", "schedule_tiles",
            "host_staging_bytes", "AttnJvpError", "TEACHER_FORCING", "BLOCK_CAUSAL"]
 
 _DT = {torch.bfloat16: _abi.DTYPE_BF16, torch.float32: _abi.DTYPE_F32}
@@ -162,6 +163,41 @@ def attn_jvp_bwd_groups(q, k, v, o, do, lse, groups: Sequence[Tuple[int, int, in
                                      dv.data_ptr(), _stream_handle(q.device))
     _abi.check(rc, "attn_jvp_bwd_groups")
     return dq, dk, dv
+
+
+def rope(q, k, tq, tk, cos, sin, out=None):
+    """Rotary position embedding of q, k and their tangents tq, tk
+    ([B, L, H, d] CUDA tensors) by per-token angles: cos, sin are fp32 [L, d/2]
+    tables. Returns the four rotated tensors (`out` may be the inputs
+    themselves, for an in-place rotation)."""
+    for t in (q, k, tq, tk):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("inputs must be contiguous CUDA tensors")
+        if t.shape != q.shape or t.dtype != q.dtype or t.device != q.device:
+            raise ValueError("q, k, tq, tk must share shape, dtype and device")
+    B, L, H, d = q.shape
+    for t in (cos, sin):
+        if t.shape != (L, d // 2) or t.dtype != torch.float32 or t.device != q.device \
+                or not t.is_contiguous():
+            raise ValueError("cos and sin must be contiguous fp32 [L, d/2] on the inputs' device")
+    shape = _shape(q, None)
+    if out is None:
+        out = tuple(torch.empty_like(q) for _ in range(4))
+    lib = _abi.load()
+    with torch.cuda.device(q.device):
+        rc = lib.attn_jvp_rope(ctypes.byref(shape), q.data_ptr(), k.data_ptr(), tq.data_ptr(),
+                               tk.data_ptr(), cos.data_ptr(), sin.data_ptr(),
+                               *(t.data_ptr() for t in out), _stream_handle(q.device))
+    _abi.check(rc, "attn_jvp_rope")
+    return out
+
+
+def attn_jvp_rope(q, k, v, tq, tk, tv, cos, sin, mode: int, chunk_tokens: int, n_chunks: int,
+                  scale: Optional[float] = None):
+    """The attention JVP with RoPE applied to the queries and keys (and their
+    tangents) first: one rotation pass, then attn_jvp on the rotated tensors."""
+    qr, kr, tqr, tkr = rope(q, k, tq, tk, cos, sin)
+    return attn_jvp(qr, kr, v, tqr, tkr, tv, mode, chunk_tokens, n_chunks, scale)
 
 
 def host_staging_bytes(B: int, L: int, H: int, d: int, dtype: torch.dtype) -> int:

@@ -103,6 +103,9 @@ def load(path: str = None) -> ctypes.CDLL:
                                             ctypes.POINTER(Group), ctypes.c_int32, vp, vp, vp,
                                             vp]
         lib.attn_jvp_bwd_groups.restype = ctypes.c_int
+        lib.attn_jvp_rope.argtypes = [ctypes.POINTER(Shape), vp, vp, vp, vp, vp, vp, vp, vp,
+                                      vp, vp, vp]
+        lib.attn_jvp_rope.restype = ctypes.c_int
         lib.attn_jvp_version.argtypes = []
         lib.attn_jvp_version.restype = ctypes.c_int32
         _lib = lib

@@ -74,10 +74,10 @@ def load_peaks():
 
 def kernel_source_hash() -> str:
     """Hash of the sources the forward kernels are built from (the backward's
-    own source file does not change them)."""
+    and the rotary embedding's own source files do not change them)."""
     h = hashlib.sha256()
     for p in sorted(glob.glob(os.path.join(ROOT, "attention_jvp_attn_b200", "csrc", "*"))):
-        if os.path.basename(p).startswith("attn_jvp_bwd"):
+        if os.path.basename(p).startswith(("attn_jvp_bwd", "attn_jvp_rope")):
             continue
         with open(p, "rb") as f:
             h.update(os.path.basename(p).encode())
@@ -506,6 +506,61 @@ def run_backward(args) -> int:
     return 0
 
 
+def run_rope(args) -> int:
+    """Rotary embedding of Q, K, tQ, tK (attn_jvp_rope) on one GPU: one JSON
+    line with the CUDA-event median over `--steps` calls after `--warmup`,
+    inputs resident (4 x the workload's tensor bytes, larger than L2). The
+    kernel is HBM-bound: algorithmic bytes are the four tensors read and
+    written plus the cos/sin tables read once."""
+    import numpy as np
+    import torch
+    import attention_jvp_attn_b200 as aj
+    from attention_jvp_attn_b200 import inputs as wl
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        raise SystemExit("--rope runs on one GPU")
+    dev = torch.device("cuda", 0)
+    w = workload_by_name(args.workload, args.heads)
+    x = wl.make_inputs(w, device=dev)
+    phi = np.random.default_rng(0).uniform(-np.pi, np.pi, (w.L, w.d // 2))
+    cos = torch.from_numpy(np.cos(phi).astype(np.float32)).to(dev)
+    sin = torch.from_numpy(np.sin(phi).astype(np.float32)).to(dev)
+    ins = (x["q"], x["k"], x["tq"], x["tk"])
+    out = tuple(torch.empty_like(t) for t in ins)
+
+    def step():
+        aj.rope(*ins, cos, sin, out=out)
+
+    for _ in range(max(args.warmup, 1)):
+        step()
+    if aj.sync_status(dev) != 0:
+        raise SystemExit("device status error")
+    clocks = ClockSampler(0)
+    clocks.start()
+    ms = []
+    for _ in range(args.steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        step()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        ms.append(e0.elapsed_time(e1))
+    ck = clocks.stop()
+    ms.sort()
+    med = ms[len(ms) // 2]
+    tensor_bytes = ins[0].numel() * ins[0].element_size()
+    alg = 8 * tensor_bytes + 2 * cos.numel() * 4
+    peaks, kind = load_peaks()
+    gbs = alg / (med * 1e-3) / 1e9
+    print(json.dumps({"mode": "rope", "workload": w.name, "dtype": w.dtype, "B": w.B, "H": w.H,
+                      "L": w.L, "d": w.d, "steps": args.steps, "warmup": args.warmup,
+                      "ms": med, "ms_min": ms[0], "ms_max": ms[-1],
+                      "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                                   "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                                   "algorithmic_bytes": alg, "peak_kind": kind},
+                      "clocks": ck}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -523,6 +578,8 @@ def main():
                     help="time every sweep point (config 5) on one GPU, one JSON line each")
     ap.add_argument("--backward", action="store_true",
                     help="time the backward of the primal attention on one GPU (one JSON line)")
+    ap.add_argument("--rope", action="store_true",
+                    help="time the rotary embedding of Q, K, tQ, tK on one GPU (one JSON line)")
     args = ap.parse_args()
     if args.warmup < 0 or args.steps < 1:
         raise SystemExit("need --steps >= 1 and --warmup >= 0")
@@ -532,6 +589,8 @@ def main():
         return run_sweep(args)
     if args.backward:
         return run_backward(args)
+    if args.rope:
+        return run_rope(args)
     return run_gpu(args)
 
 

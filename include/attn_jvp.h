@@ -290,6 +290,40 @@ int attn_jvp_bwd_groups(const attn_jvp_shape* shape,
                         void* dq, void* dk, void* dv,
                         void* stream);
 
+/* ---- rotary position embedding ahead of the attention ------------------ */
+
+/*
+ * attn_jvp_rope - rotary position embedding of q, k and their tangents tq, tk
+ * (Causal-rCM summary page, section 3, "KV Cache": RoPE is the positional
+ * treatment of queries and keys, one of the attention's neighbours in the
+ * layer-level JVP). The pages give no formula; this is the standard rotary
+ * embedding on adjacent pairs, with per-token angles phi supplied as tables:
+ *
+ *     x'_2i   = x_2i cos(phi_ti) - x_2i+1 sin(phi_ti)
+ *     x'_2i+1 = x_2i sin(phi_ti) + x_2i+1 cos(phi_ti)
+ *
+ * for every batch and head of token t. The rotation does not depend on its
+ * input, so the tangents of the rotated queries and keys are the rotated
+ * tangents; attn_jvp_fwd on the four outputs (with v and tv unchanged) is the
+ * attention JVP with RoPE in front.
+ *
+ *   shape              as for attn_jvp_fwd (dtype, d; scale unused)
+ *   q, k, tq, tk       device inputs, [B, L, H, d] of shape->dtype
+ *   cos, sin           device tables, [L, d/2] float (token t, pair i)
+ *   q_out .. tk_out    device outputs, [B, L, H, d] of shape->dtype; each may be
+ *                      its own input (in place), and must not overlap any other
+ *   stream             cudaStream_t to launch on
+ *
+ * All pointers 16-byte aligned. Arithmetic is fp32; bf16 outputs are rounded
+ * to nearest even. One launch, one pass over HBM. Returns ATTN_JVP_OK after
+ * enqueueing, or an error code with nothing launched; does not synchronize.
+ */
+int attn_jvp_rope(const attn_jvp_shape* shape,
+                  const void* q, const void* k, const void* tq, const void* tk,
+                  const float* cos, const float* sin,
+                  void* q_out, void* k_out, void* tq_out, void* tk_out,
+                  void* stream);
+
 /* ---- host-side helpers (need no GPU) ---------------------------------- */
 
 /* Number of admissible (query, key) pairs per (batch, head):

@@ -18,6 +18,10 @@ one for O and tO, one for LSE, on the process group's backend (NCCL over
 NVLink between GPUs; gloo in the CPU tests). The attention itself is the
 library's kernel; `attn` can be replaced (the tests put the float64 oracle
 there to check the data movement exactly).
+
+The backward (ulysses_attn_jvp_bwd) is the transposed exchange: Q, K, V, O,
+dO and LSE go to head shards, the library's backward runs on the shard, and
+dQ, dK, dV go back to sequence blocks (`bwd` can be replaced likewise).
 """
 from __future__ import annotations
 
@@ -65,6 +69,18 @@ def _lse_to_seq(lse: Tensor, G: int, group) -> Tensor:
     return recv.permute(1, 0, 2, 3).reshape(B, G * Hg, Ls)
 
 
+def _lse_to_heads(lse: Tensor, G: int, group) -> Tensor:
+    """[B, H, L/G] -> [B, H/G, L] (the inverse of _lse_to_seq)."""
+    B, H, Ls = lse.shape
+    Hg = H // G
+    # chunk for destination rank j: heads [j Hg, (j+1) Hg)
+    send = lse.reshape(B, G, Hg, Ls).permute(1, 0, 2, 3).contiguous()
+    recv = torch.empty_like(send)
+    dist.all_to_all_single(recv, send, group=group)
+    # recv[s] is sequence block s of my heads
+    return recv.permute(1, 2, 0, 3).reshape(B, Hg, G * Ls)
+
+
 def _kernel_attn(mask):
     from . import attn_jvp, attn_jvp_groups
 
@@ -107,3 +123,55 @@ def ulysses_attn_jvp(q: Tensor, k: Tensor, v: Tensor, tq: Tensor, tk: Tensor, tv
     o, to, lse = run(qh, kh, vh, tqh, tkh, tvh, scale)
     out = _heads_to_seq(torch.stack((o, to)), G, group)
     return out[0], out[1], _lse_to_seq(lse.contiguous(), G, group)
+
+
+def _kernel_bwd(mask):
+    from . import attn_jvp_bwd, attn_jvp_bwd_groups
+
+    def run(q, k, v, o, do, lse, scale, dlse):
+        if isinstance(mask, dict):
+            return attn_jvp_bwd_groups(q, k, v, o, do, lse, mask["groups"], scale, dlse=dlse)
+        mode, c, n = mask
+        return attn_jvp_bwd(q, k, v, o, do, lse, mode, c, n, scale, dlse=dlse)
+
+    return run
+
+
+def ulysses_attn_jvp_bwd(q: Tensor, k: Tensor, v: Tensor, o: Tensor, do: Tensor, lse: Tensor,
+                         mask, scale: Optional[float] = None, dlse: Optional[Tensor] = None,
+                         group=None, bwd: Optional[Callable[..., Tuple[Tensor, Tensor, Tensor]]] = None
+                         ) -> Tuple[Tensor, Tensor, Tensor]:
+    """dQ, dK, dV ([B, L/G, H, d]) of this rank's sequence block, for the
+    attention that ulysses_attn_jvp computed: the transposed exchange of the
+    forward. q, k, v, o, do are this rank's sequence blocks; lse (and dlse, if
+    given) are [B, H, L/G] as ulysses_attn_jvp returns them. One all-to-all
+    takes the five tensors to head shards over the full sequence, one takes
+    LSE (and one dLSE); the backward runs on the head shard, and one
+    all-to-all returns dQ, dK, dV to sequence blocks. Ulysses has no partial
+    sums: every gradient row is computed whole on one rank."""
+    G = dist.get_world_size(group)
+    B, Ls, H, d = q.shape
+    for t in (k, v, o, do):
+        if t.shape != q.shape or t.dtype != q.dtype or t.device != q.device:
+            raise ValueError("q, k, v, o, do must share shape, dtype and device")
+    if H % G:
+        raise ValueError(f"heads ({H}) must be a multiple of the group size ({G})")
+    for t in (lse,) + ((dlse,) if dlse is not None else ()):
+        if t.shape != (B, H, Ls):
+            raise ValueError("lse and dlse must be [B, H, L/G]")
+    L = Ls * G
+    if isinstance(mask, dict):
+        if int(mask["groups"][-1][0]) != L:
+            raise ValueError("the group table does not cover the gathered sequence")
+    else:
+        mode, c, n = mask
+        if (2 if mode == _wl.TEACHER_FORCING else 1) * n * c != L:
+            raise ValueError("the mask's sequence length differs from G x the local block")
+    run = bwd if bwd is not None else _kernel_bwd(mask)
+    full = _seq_to_heads(torch.stack((q, k, v, o, do)), G, group)
+    qh, kh, vh, oh, doh = (t.contiguous() for t in full.unbind(0))
+    lse_h = _lse_to_heads(lse.contiguous(), G, group).contiguous()
+    dlse_h = _lse_to_heads(dlse.contiguous(), G, group).contiguous() if dlse is not None else None
+    dq, dk, dv = run(qh, kh, vh, oh, doh, lse_h, scale, dlse_h)
+    out = _heads_to_seq(torch.stack((dq, dk, dv)), G, group)
+    return out[0], out[1], out[2]

@@ -1,4 +1,5 @@
-"""Tangent-aware Ulysses exchange (seq -> heads -> seq) on CPU ranks (gloo).
+"""Tangent-aware Ulysses exchange (seq -> heads -> seq) on CPU ranks (gloo),
+for the attention JVP and for the backward of the primal attention.
 
 Each rank holds one sequence block of Q, K, V, tQ, tK, tV; after the
 exchange it runs the attention JVP for its heads over the full sequence and
@@ -109,6 +110,107 @@ def test_ulysses_exchange_matches_unsharded_oracle(name):
         assert np.array_equal(o, O[:, r * Ls:(r + 1) * Ls])
         assert np.array_equal(to, tO[:, r * Ls:(r + 1) * Ls])
         assert np.array_equal(lse, LSE[:, :, r * Ls:(r + 1) * Ls])
+
+
+def _mask_matrix(mask):
+    from oracle import attn_jvp_oracle as orc
+    if isinstance(mask, dict):
+        return orc.mask_matrix_groups(mask["groups"])
+    return orc.mask_matrix(*mask)
+
+
+def _lse_based_bwd(mask):
+    """Float64 backward that, like the kernel, rebuilds P from the LSE it is
+    given and takes D_i from the O it is given, so a misplaced O or LSE row
+    changes the result. Per (batch, head) 2-D products: the same bits whatever
+    heads a rank holds."""
+    M = _mask_matrix(mask)
+
+    def run(q, k, v, o, do, lse, scale, dlse):
+        B, L, H, d = q.shape
+        s = 1.0 / np.sqrt(d) if scale is None else scale
+        outs = [np.zeros((B, L, H, d)) for _ in range(3)]
+        for b in range(B):
+            for h in range(H):
+                qq, kk, vv, oo, dd = (t[b, :, h].numpy() for t in (q, k, v, o, do))
+                P = np.where(M, np.exp(s * (qq @ kk.T) - lse[b, h].numpy()[:, None]), 0.0)
+                D = (dd * oo).sum(axis=1) - (dlse[b, h].numpy() if dlse is not None else 0.0)
+                dS = P * (dd @ vv.T - D[:, None])
+                outs[0][b, :, h] = s * (dS @ kk)
+                outs[1][b, :, h] = s * (dS.T @ qq)
+                outs[2][b, :, h] = P.T @ dd
+        return tuple(torch.from_numpy(t) for t in outs)
+
+    return run
+
+
+def _bwd_full(case):
+    from oracle import attn_jvp_oracle as orc
+    B, L, H, d, mask, scale, seed = case
+    q, k, v, do, _, _ = _full_inputs(B, L, H, d, seed)
+    if isinstance(mask, dict):
+        O, LSE = orc.attn_forward_dense(q, k, v, 0, 1, 1, scale, groups=mask["groups"])
+    else:
+        O, LSE = orc.attn_forward_dense(q, k, v, *mask, scale)
+    dlse = torch.randn((B, H, L), generator=torch.Generator().manual_seed(seed + 1),
+                       dtype=torch.float64)
+    return q, k, v, torch.from_numpy(O), do, torch.from_numpy(LSE), dlse
+
+
+def _bwd_worker(rank, world, port, case, q):
+    import datetime
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from attention_jvp_attn_b200.ulysses import ulysses_attn_jvp_bwd
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        B, L, H, d, mask, scale, seed = case
+        qq, k, v, o, do, lse, dlse = _bwd_full(case)
+        Ls = L // world
+        sl = slice(rank * Ls, (rank + 1) * Ls)
+        local = [t[:, sl].contiguous() for t in (qq, k, v, o, do)]
+        out = ulysses_attn_jvp_bwd(*local, lse[:, :, sl].contiguous(), mask, scale,
+                                   dlse=dlse[:, :, sl].contiguous(), bwd=_lse_based_bwd(mask))
+        q.put((rank,) + tuple(t.numpy() for t in out))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_ulysses_backward_matches_unsharded(name):
+    from oracle import attn_jvp_oracle as orc
+    world = WORLD[name]
+    case = CASES[name]
+    B, L, H, d, mask, scale, seed = case
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_bwd_worker, args=(r, world, port, case, q))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    res = {}
+    for _ in range(world):
+        r, *g = q.get(timeout=120)
+        res[r] = g
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    qq, k, v, o, do, lse, dlse = _bwd_full(case)
+    whole = [t.numpy() for t in _lse_based_bwd(mask)(qq, k, v, o, do, lse, scale, dlse)]
+    groups = mask["groups"] if isinstance(mask, dict) else None
+    m = (0, 1, 1) if groups else mask
+    ref = orc.attn_vjp_dense(qq, k, v, do, *m, scale, dlse=dlse.numpy(), groups=groups)
+    Ls = L // world
+    for r in range(world):
+        for got, full, exact in zip(res[r], whole, ref):
+            # bit-equal to the same backward on the unsharded problem
+            assert np.array_equal(got, full[:, r * Ls:(r + 1) * Ls])
+            # and equal to the oracle's VJP up to float64 rounding
+            np.testing.assert_allclose(got, exact[:, r * Ls:(r + 1) * Ls], rtol=1e-9, atol=1e-11)
 
 
 def test_ulysses_rejects_a_mask_of_another_length():

@@ -271,6 +271,74 @@ def attn_vjp_rows(q, k, v, do, mode: int, c: int, n: int, scale: Optional[float]
     return dQ, dK, dV
 
 
+def _vjp_row_block(q, k, v, do, M, s, rr, dlse):
+    """P, dP and D (= rowsum(P * dP) - dLSE) of the query rows rr over all
+    keys, with M the [len(rr), L] admissible pattern."""
+    S = np.where(M, s * (q[rr] @ k.T), -np.inf)
+    smax = S.max(axis=1, keepdims=True)
+    lse = smax[:, 0] + np.log(np.exp(S - smax).sum(axis=1))
+    P = np.exp(S - lse[:, None])
+    dP = do[rr] @ v.T
+    D = (P * dP).sum(axis=1)
+    if dlse is not None:
+        D = D - dlse[rr]
+    return P, dP, D
+
+
+def attn_vjp_dq_rows(q, k, v, do, mode: int, c: int, n: int, scale: Optional[float],
+                     rows: Sequence[int], dlse=None, groups: Optional[Sequence[Group]] = None,
+                     block: int = 64) -> np.ndarray:
+    """dQ [R, d] for the given query rows of ONE (batch, head): the rows of
+    attn_vjp_rows' dQ, each from its own row of P (the same definition; only
+    the rows asked for are formed). dlse, if given, is the [L] cotangent."""
+    q, k, v, do = (_as64(x) for x in (q, k, v, do))
+    dl = None if dlse is None else _as64(dlse)
+    L, d = q.shape
+    s = (1.0 / math.sqrt(d)) if scale is None else float(scale)
+    rows = np.asarray(rows, dtype=np.int64)
+    keys = np.arange(L)
+    out = np.empty((rows.shape[0], d))
+    for r0 in range(0, rows.shape[0], block):
+        rr = rows[r0:r0 + block]
+        M = allowed_groups(groups, rr[:, None], keys[None, :]) if groups is not None \
+            else allowed(mode, c, n, rr[:, None], keys[None, :])
+        P, dP, D = _vjp_row_block(q, k, v, do, M, s, rr, dl)
+        out[r0:r0 + block] = s * ((P * (dP - D[:, None])) @ k)
+    return out
+
+
+def attn_vjp_dkdv_cols(q, k, v, do, mode: int, c: int, n: int, scale: Optional[float],
+                       cols: Sequence[int], dlse=None, groups: Optional[Sequence[Group]] = None,
+                       block: int = 256) -> Tuple[np.ndarray, np.ndarray]:
+    """dK, dV [C, d] for the given key columns of ONE (batch, head): column j
+    sums over the rows that may attend to key j, each row's P and D taken
+    from that whole row (the same definition as attn_vjp_rows, only the
+    columns asked for are formed). Cost grows with the number of rows that
+    attend to the columns."""
+    q, k, v, do = (_as64(x) for x in (q, k, v, do))
+    dl = None if dlse is None else _as64(dlse)
+    L, d = q.shape
+    s = (1.0 / math.sqrt(d)) if scale is None else float(scale)
+    cols = np.asarray(cols, dtype=np.int64)
+    keys = np.arange(L)
+    t = np.arange(L)
+    seen = allowed_groups(groups, t[:, None], cols[None, :]) if groups is not None \
+        else allowed(mode, c, n, t[:, None], cols[None, :])
+    rows = np.nonzero(seen.any(axis=1))[0]
+    dK = np.zeros((cols.shape[0], d))
+    dV = np.zeros((cols.shape[0], d))
+    for r0 in range(0, rows.shape[0], block):
+        rr = rows[r0:r0 + block]
+        M = allowed_groups(groups, rr[:, None], keys[None, :]) if groups is not None \
+            else allowed(mode, c, n, rr[:, None], keys[None, :])
+        P, dP, D = _vjp_row_block(q, k, v, do, M, s, rr, dl)
+        Pc = P[:, cols]
+        dSc = Pc * (dP[:, cols] - D[:, None])
+        dV += Pc.T @ do[rr]
+        dK += s * (dSc.T @ q[rr])
+    return dK, dV
+
+
 def attn_vjp_dense(q, k, v, do, mode: int, c: int, n: int, scale: Optional[float] = None,
                    dlse=None, groups: Optional[Sequence[Group]] = None):
     """dQ, dK, dV [B, L, H, d] for [B, L, H, d] inputs and output cotangent dO

@@ -166,6 +166,29 @@ def test_lse_cotangent_on_a_zero_query():
     assert not dK.any() and not dV.any()
 
 
+@pytest.mark.parametrize("case", CASES, ids=_ids)
+def test_sampled_rows_and_columns_match_the_dense_backward(case):
+    # the row- and column-sampled forms used on large workloads give the same
+    # numbers as the pinned dense backward
+    mode, c, n, d, H, scale, groups = case
+    M = _mask(mode, c, n, groups)
+    L = M.shape[0]
+    q, k, v, do = _rand(L, H, d, seed=L * 5 + d)
+    dlse = np.random.default_rng(L + 1).standard_normal((1, H, L))
+    dQ, dK, dV = orc.attn_vjp_dense(q, k, v, do, mode, c, n, scale, dlse=dlse, groups=groups)
+    rng = np.random.default_rng(2)
+    rows = np.unique(np.concatenate([[0, L - 1], rng.integers(0, L, 5)]))
+    cols = np.unique(np.concatenate([[0, L - 1], rng.integers(0, L, 5)]))
+    for h in range(H):
+        a = orc.attn_vjp_dq_rows(q[0, :, h], k[0, :, h], v[0, :, h], do[0, :, h], mode, c, n,
+                                 scale, rows, dlse=dlse[0, h], groups=groups, block=3)
+        np.testing.assert_allclose(a, dQ[0, rows, h], rtol=1e-12, atol=1e-13)
+        bk, bv = orc.attn_vjp_dkdv_cols(q[0, :, h], k[0, :, h], v[0, :, h], do[0, :, h], mode, c,
+                                        n, scale, cols, dlse=dlse[0, h], groups=groups, block=4)
+        np.testing.assert_allclose(bk, dK[0, cols, h], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(bv, dV[0, cols, h], rtol=1e-12, atol=1e-13)
+
+
 # ---------------------------------------------------------------------------
 # Planted mistakes: each must fail at least one pin above.
 

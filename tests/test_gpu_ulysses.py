@@ -1,6 +1,7 @@
-"""The Ulysses path on a GPU with the library's kernel as the local attention
-(NCCL process group of one rank: the exchange is the identity, the kernel and
-the layout code are the real ones). Its outputs must equal a direct call's.
+"""The Ulysses path on a GPU with the library's kernels as the local attention
+and backward (NCCL process group of one rank: the exchange is the identity,
+the kernels and the layout code are the real ones). Its outputs must equal a
+direct call's, bit for bit.
 """
 import datetime
 import os
@@ -12,7 +13,7 @@ import torch.distributed as dist
 
 import attention_jvp_attn_b200 as aj
 from attention_jvp_attn_b200 import inputs as wl
-from attention_jvp_attn_b200.ulysses import ulysses_attn_jvp
+from attention_jvp_attn_b200.ulysses import ulysses_attn_jvp, ulysses_attn_jvp_bwd
 
 pytestmark = pytest.mark.gpu
 
@@ -44,3 +45,21 @@ def test_ulysses_single_rank_equals_direct_call(cuda_device, nccl_group, d):
     assert aj.sync_status() == 0
     for u, v in zip(a, b):
         assert torch.equal(u.view(torch.uint8), v.contiguous().view(torch.uint8))
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_ulysses_backward_single_rank_equals_direct_call(cuda_device, nccl_group, d):
+    w = wl.Workload("ulysses_bwd", B=1, H=4, d=d, n_chunks=3, chunk_tokens=150,
+                    mode=wl.BLOCK_CAUSAL, seed=516)
+    x = wl.make_inputs(w, device=cuda_device)
+    q, k, v = x["q"], x["k"], x["v"]
+    m = (w.mode, w.chunk_tokens, w.n_chunks)
+    o, _, lse = aj.attn_jvp(q, k, v, x["tq"], x["tk"], x["tv"], *m)
+    g = torch.Generator(device=cuda_device).manual_seed(7)
+    do = torch.randn(q.shape, generator=g, device=cuda_device).to(q.dtype)
+    a = aj.attn_jvp_bwd(q, k, v, o, do, lse, *m)
+    b = ulysses_attn_jvp_bwd(q, k, v, o, do, lse, m)
+    torch.cuda.synchronize()
+    assert aj.sync_status() == 0
+    for u, v2 in zip(a, b):
+        assert torch.equal(u.view(torch.uint8), v2.contiguous().view(torch.uint8))

@@ -189,6 +189,35 @@ def test_sampled_rows_and_columns_match_the_dense_backward(case):
         np.testing.assert_allclose(bv, dV[0, cols, h], rtol=1e-12, atol=1e-13)
 
 
+def _golden_cases():
+    import json
+    import os
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "vjp_closed_form.json")
+    with open(path) as f:
+        return json.load(f)["cases"]
+
+
+def _g(x):
+    if isinstance(x, list):
+        return [_g(y) for y in x]
+    if isinstance(x, str):
+        return float(eval(x, {"__builtins__": {}}, {"ln2": math.log(2), "ln3": math.log(3)}))
+    return float(x)
+
+
+@pytest.mark.parametrize("case", _golden_cases(), ids=lambda c: c["name"])
+def test_hand_derived_cases(case):
+    # tests/golden/vjp_closed_form.json: gradients derived by hand
+    t = {k: np.array(_g(case[k])) for k in ("q", "k", "v", "do", "dQ", "dK", "dV")}
+    dlse = np.array(_g(case["dlse"])) if "dlse" in case else None
+    dQ, dK, dV = orc.attn_vjp_rows(t["q"], t["k"], t["v"], t["do"], case["mode"],
+                                   case["chunk_tokens"], case["n_chunks"], case["scale"],
+                                   dlse=dlse)
+    np.testing.assert_allclose(dQ, t["dQ"], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(dK, t["dK"], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(dV, t["dV"], rtol=0, atol=1e-14)
+
+
 # ---------------------------------------------------------------------------
 # Planted mistakes: each must fail at least one pin above.
 
@@ -223,6 +252,7 @@ PIN_CHECKS = (
        lambda: test_finite_differences_of_a_scalar_loss(BC),
        test_one_admissible_key_per_row, test_zero_cotangent_gives_zero_gradients,
        test_lse_cotangent_on_a_zero_query]
+    + [lambda c=c: test_hand_derived_cases(c) for c in _golden_cases()]
 )
 
 

@@ -226,3 +226,31 @@ def test_ulysses_rejects_a_mask_of_another_length():
             ulysses_attn_jvp(*x, (1, 2, 3), None, attn=_oracle_attn((1, 2, 3)))  # L=8 vs 6
     finally:
         dist.destroy_process_group()
+
+
+def test_ulysses_backward_rejects_bad_arguments():
+    import torch.distributed as dist
+    from attention_jvp_attn_b200.ulysses import ulysses_attn_jvp_bwd
+    port = _free_port()
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=0, world_size=1)
+    try:
+        mask = (1, 2, 3)  # block causal, L = 6
+        x = [torch.zeros(1, 6, 3, 4, dtype=torch.float64) for _ in range(5)]
+        lse = torch.zeros(1, 3, 6, dtype=torch.float64)
+        bwd = _lse_based_bwd(mask)
+        with pytest.raises(ValueError):  # LSE of another length
+            ulysses_attn_jvp_bwd(*x, torch.zeros(1, 3, 5, dtype=torch.float64), mask, bwd=bwd)
+        with pytest.raises(ValueError):  # dLSE of another shape
+            ulysses_attn_jvp_bwd(*x, lse, mask, dlse=torch.zeros(1, 2, 6, dtype=torch.float64),
+                                 bwd=bwd)
+        with pytest.raises(ValueError):  # mask of another length
+            ulysses_attn_jvp_bwd(*x, lse, (1, 2, 2), bwd=bwd)
+        with pytest.raises(ValueError):  # inputs of different shapes
+            ulysses_attn_jvp_bwd(*x[:4], torch.zeros(1, 6, 3, 5, dtype=torch.float64), lse, mask,
+                                 bwd=bwd)
+        out = ulysses_attn_jvp_bwd(*x, lse, mask, bwd=bwd)  # and the valid call runs
+        assert all(t.shape == (1, 6, 3, 4) for t in out)
+    finally:
+        dist.destroy_process_group()

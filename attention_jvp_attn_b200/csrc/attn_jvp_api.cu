@@ -9,10 +9,7 @@
 #include <cstring>
 #include <functional>
 #include <mutex>
-#include <numeric>
-#include <queue>
 #include <utility>
-#include <vector>
 
 #include "attn_jvp.h"
 #include "kernels.cuh"
@@ -215,15 +212,19 @@ void set_mask(MaskSpec* dst, ajvp::GroupRange* dst_groups, const MaskSpec& ms) {
   dst->groups = nullptr;  // the kernels point it at their own parameter copy
 }
 
-// Query row blocks (of `bm` rows) of one head, most key tiles first (stable among equals).
+// Query row blocks (of `bm` rows) of one head, most key tiles first (ties:
+// lower block first, the order a stable sort gives). Host scratch is fixed
+// thread-local arrays: building the order allocates nothing.
 int fill_order(const MaskSpec& ms, int n_qtiles, int bm, uint16_t* order) {
   if (n_qtiles > ajvp::kMaxOrder) return 0;
-  std::vector<int> cost(n_qtiles), idx(n_qtiles);
+  static thread_local int cost[ajvp::kMaxOrder];
+  static thread_local int idx[ajvp::kMaxOrder];
   for (int t = 0; t < n_qtiles; ++t) {
     cost[t] = ajvp::make_tile_sched(ms, t, bm, ajvp::kTcBlockN).count();
     idx[t] = t;
   }
-  std::stable_sort(idx.begin(), idx.end(), [&](int a, int b) { return cost[a] > cost[b]; });
+  std::sort(idx, idx + n_qtiles,
+            [&](int a, int b) { return cost[a] != cost[b] ? cost[a] > cost[b] : a < b; });
   for (int r = 0; r < n_qtiles; ++r) order[r] = static_cast<uint16_t>(idx[r]);
   return n_qtiles;
 }
@@ -232,33 +233,42 @@ int fill_order(const MaskSpec& ms, int n_qtiles, int bm, uint16_t* order) {
 // running units share a head's keys in L2), each query block of the head goes,
 // longest first, to the unit with the least work so far (ties: lowest unit).
 // Work is the block's key-tile count. Returns false if the lists do not fit.
+// The min-heap of unit loads and the per-item assignment live in fixed
+// thread-local arrays: no host allocation per call.
 bool fill_work_lists(const MaskSpec& ms, int bh_count, int n_qtiles, int bm, int units,
                      const uint16_t* head_order, uint16_t* lists, uint16_t* unit_start) {
   const int n_items = bh_count * n_qtiles;
   if (n_items > ajvp::kMaxOrder || units < 1 || units > ajvp::kMaxUnits) return false;
-  std::vector<int> cost(n_qtiles);
+  static thread_local int cost[ajvp::kMaxOrder];
+  static thread_local uint16_t item_pos[ajvp::kMaxOrder];  // assignment order: item position
+  static thread_local uint16_t item_unit[ajvp::kMaxOrder];  // and its unit
+  static thread_local std::pair<int64_t, int> heap[ajvp::kMaxUnits];  // (work so far, unit)
   for (int t = 0; t < n_qtiles; ++t)
     cost[t] = ajvp::make_tile_sched(ms, t, bm, ajvp::kTcBlockN).count();
-  using Load = std::pair<int64_t, int>;  // (work so far, unit)
-  std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
-  for (int u = 0; u < units; ++u) heap.push({0, u});
-  std::vector<std::vector<uint16_t>> per(units);
+  // min-heap on (work, unit): the comparator is "greater"
+  const auto cmp = std::greater<std::pair<int64_t, int>>();
+  for (int u = 0; u < units; ++u) heap[u] = {0, u};
+  std::make_heap(heap, heap + units, cmp);
+  int a = 0;
   for (int bh = 0; bh < bh_count; ++bh) {
     for (int r = 0; r < n_qtiles; ++r) {
       const int qt = head_order ? head_order[r] : n_qtiles - 1 - r;
-      Load x = heap.top();
-      heap.pop();
-      per[x.second].push_back(static_cast<uint16_t>(bh * n_qtiles + qt));
+      std::pop_heap(heap, heap + units, cmp);
+      std::pair<int64_t, int>& x = heap[units - 1];
+      item_pos[a] = static_cast<uint16_t>(bh * n_qtiles + qt);
+      item_unit[a] = static_cast<uint16_t>(x.second);
+      ++a;
       x.first += cost[qt];
-      heap.push(x);
+      std::push_heap(heap, heap + units, cmp);
     }
   }
-  int at = 0;
-  for (int u = 0; u < units; ++u) {
-    unit_start[u] = static_cast<uint16_t>(at);
-    for (uint16_t pos : per[u]) lists[at++] = pos;
-  }
-  unit_start[units] = static_cast<uint16_t>(at);
+  // Lists in unit order, each unit's items in assignment order.
+  for (int u = 0; u <= units; ++u) unit_start[u] = 0;
+  for (int i = 0; i < n_items; ++i) ++unit_start[item_unit[i] + 1];
+  for (int u = 0; u < units; ++u) unit_start[u + 1] += unit_start[u];
+  static thread_local uint16_t fill[ajvp::kMaxUnits];
+  for (int u = 0; u < units; ++u) fill[u] = unit_start[u];
+  for (int i = 0; i < n_items; ++i) lists[fill[item_unit[i]]++] = item_pos[i];
   return true;
 }
 
@@ -600,12 +610,12 @@ int attn_jvp_fwd_noalloc(const attn_jvp_shape* shape, const void* q, const void*
   rc = launch_bf16(&launch_state, shape, q, k, v, tq, tk, tv, mask_spec(mask, shape->L), o, to, lse,
                    s);
   if (rc != ATTN_JVP_OK) return rc;
-  if (cudaStreamSynchronize(s) != cudaSuccess) {
-    cudaGetLastError();
-    return ATTN_JVP_ERR_CUDA;
-  }
+  // The word is read back on the same stream (not the legacy default stream),
+  // then one wait for the stream covers the kernel and the copy.
   unsigned int word = 0;
-  if (cudaMemcpy(&word, st->scratch, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) {
+  if (cudaMemcpyAsync(&word, st->scratch, sizeof(word), cudaMemcpyDeviceToHost, s) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess) {
     cudaGetLastError();
     return ATTN_JVP_ERR_CUDA;
   }

@@ -190,6 +190,28 @@ def workload_config(w, n_gpus):
 
 # --------------------------------------------------------------------------- oracle timing
 
+def _oracle_threads() -> int:
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max((i.get("num_threads", 1) for i in info), default=1)
+    except Exception:
+        return 1
+
+
+def _timed_oracle_rows(w, x64, rows):
+    """The float64 oracle on query rows `rows` of one (batch, head) whose [L, d]
+    inputs are x64: (O, tO, LSE of the rows, seconds, admissible pairs)."""
+    import numpy as np
+    from oracle import attn_jvp_oracle as orc
+    rows = np.asarray(rows, dtype=np.int64)
+    t0 = time.perf_counter()
+    O, tO, lse = orc.attn_jvp_rows(*x64, w.mode, w.chunk_tokens, w.n_chunks, w.scale, rows)
+    secs = time.perf_counter() - t0
+    M = orc.allowed(w.mode, w.chunk_tokens, w.n_chunks, rows[:, None], np.arange(w.L)[None, :])
+    return O, tO, lse, secs, int(M.sum())
+
+
 def oracle_sample(w, budget_s: float, seed: int = 0):
     """Time the float64 oracle on seeded random query rows of head 0 of the
     workload (CPU inputs drawn from the same generator recipe), growing the
@@ -197,14 +219,7 @@ def oracle_sample(w, budget_s: float, seed: int = 0):
     rows, seconds, threads)."""
     import numpy as np
     import torch
-    from attention_jvp_attn_b200 import inputs as wl
     from oracle import attn_jvp_oracle as orc
-    try:
-        import threadpoolctl
-        info = threadpoolctl.threadpool_info()
-        threads = max((i.get("num_threads", 1) for i in info), default=1)
-    except Exception:
-        threads = 1
     g = torch.Generator().manual_seed(w.seed)
     one = (w.L, w.d)
     x = [(torch.randn(one, generator=g) * s).to(torch.bfloat16 if w.dtype == "bf16" else torch.float32)
@@ -215,15 +230,75 @@ def oracle_sample(w, budget_s: float, seed: int = 0):
     batch = 16
     while total_t < budget_s:
         rows = rng.integers(0, w.L, size=batch)
-        t0 = time.perf_counter()
-        orc.attn_jvp_rows(*x64, w.mode, w.chunk_tokens, w.n_chunks, w.scale, rows)
-        total_t += time.perf_counter() - t0
-        M = orc.allowed(w.mode, w.chunk_tokens, w.n_chunks, rows[:, None], np.arange(w.L)[None, :])
-        total_pairs += int(M.sum())
+        _, _, _, t, pairs = _timed_oracle_rows(w, x64, rows)
+        total_t += t
+        total_pairs += pairs
         rows_done += batch
         if total_t < budget_s / 4:
             batch *= 2
-    return 12 * w.d * total_pairs / total_t, rows_done, total_t, threads
+    return 12 * w.d * total_pairs / total_t, rows_done, total_t, _oracle_threads()
+
+
+def oracle_check_and_time(w, x, outs, budget_s: float, seed: int = 0):
+    """The CPU-baseline leg on the timed call's own data: the float64 oracle
+    on sampled query rows of two (batch, head) slices of the GPU inputs `x`,
+    timed, and its O, tO, LSE compared with the GPU outputs `outs` of the
+    timed call on the same rows. Rows: every chunk's first and last row, the
+    rows on both sides of the 128- and 256-row tile edges around chunk
+    boundaries, the ragged tail and 64 seeded random rows per slice; then
+    seeded random rows of the first slice until about `budget_s` seconds of
+    oracle work. Returns (cpu_baseline dict, parity dict)."""
+    import numpy as np
+    from attention_jvp_attn_b200 import inputs as wl
+    from oracle import attn_jvp_oracle as orc
+    o, to, lse = outs
+    tol = 2e-2 if w.dtype == "bf16" else 1e-4
+    tol_lse = 1e-3 if w.dtype == "bf16" else 1e-4
+    struct = sorted(set(wl.sample_rows(w, n_random=64, seed=seed + 11, tile=128)) |
+                    set(wl.sample_rows(w, n_random=0, tile=256)))
+    slices = [(0, 0), (w.B - 1, w.H - 1)]
+    worst = {"O": 0.0, "tO": 0.0, "LSE": 0.0}
+    total_t, total_pairs, n_rows = 0.0, 0, 0
+    rng = np.random.default_rng(seed)
+
+    def check(b, h, x64, rows):
+        nonlocal total_t, total_pairs, n_rows
+        O, tO, L_, t, pairs = _timed_oracle_rows(w, x64, rows)
+        total_t += t
+        total_pairs += pairs
+        n_rows += len(rows)
+        idx = np.asarray(rows)
+        got = (o[b, idx, h].double().cpu().numpy(), to[b, idx, h].double().cpu().numpy(),
+               lse[b, h, idx].double().cpu().numpy())
+        for name, g, r, tl in (("O", got[0], O, tol), ("tO", got[1], tO, tol),
+                               ("LSE", got[2], L_, tol_lse)):
+            ratio = np.abs(g - r) / (tl * (1.0 + np.abs(r)))
+            worst[name] = max(worst[name], float(np.nanmax(ratio)) if np.isfinite(g).all()
+                              else float("inf"))
+
+    first = None
+    for b, h in slices:
+        x64 = [orc._as64(x[n][b, :, h]) for n in wl.TENSOR_ORDER]
+        first = first or (b, h, x64)
+        check(b, h, x64, struct)
+    b, h, x64 = first
+    batch = 16
+    while total_t < budget_s:
+        check(b, h, x64, sorted(set(rng.integers(0, w.L, size=batch).tolist())))
+        if total_t < budget_s / 4:
+            batch *= 2
+    cpu = {"value": 12 * w.d * total_pairs / total_t / 1e12, "unit": "TFLOP/s",
+           "cores": _oracle_threads(), "kind": "oracle",
+           "sample": (f"{n_rows} query rows of (batch, head) slices {slices} of the timed "
+                      f"call's inputs (chunk and tile edges, ragged tail, seeded random rows), "
+                      f"{total_t:.1f} s of float64 oracle work; effective FLOPs = 12 d x "
+                      f"admissible pairs of those rows")}
+    parity = {"rows": n_rows, "slices": [list(s) for s in slices],
+              "bound": f"|err| <= {tol} (1 + |ref|) for O and tO, {tol_lse} (1 + |ref|) for LSE",
+              "max_err_over_bound_O": worst["O"], "max_err_over_bound_tO": worst["tO"],
+              "max_err_over_bound_LSE": worst["LSE"],
+              "pass": all(v <= 1.0 for v in worst.values())}
+    return cpu, parity
 
 
 def run_reference(args):
@@ -236,18 +311,22 @@ def run_reference(args):
         oracle_sample(w, budget_s=0.5)
     vals, secs, rows_all = [], 0.0, 0
     threads = 1
+    t_steps = time.perf_counter()
     for _ in range(args.steps):
         v, rows, t, threads = oracle_sample(w, budget_s=args.ref_budget)
         vals.append(v)
         secs += t
         rows_all += rows
+    wall_s = time.perf_counter() - t_steps
     value = statistics.mean(vals) / 1e12
     sample = (f"{rows_all} seeded random query rows of head 0 over {args.steps} steps "
               f"(about {args.ref_budget:.0f} s each), float64 dense rows masked by the explicit "
               f"predicate; effective FLOPs = 12 d x admissible pairs of the sampled rows")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": 1e3 * flops_per_step(w) / (value * 1e12),
+            "ms_per_step": 1e3 * wall_s / args.steps,
+            "step": "one bounded sample of query rows of the workload (not a full call)",
+            "extrapolated_full_call_ms": 1e3 * flops_per_step(w) / (value * 1e12),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": workload_config(w, 1),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads,
@@ -332,6 +411,7 @@ def run_gpu(args):
 
     # end to end through the host-buffer C-ABI entry point (pinned host memory)
     e2e = None
+    e2e_steps = args.e2e_steps if args.e2e_steps is not None else args.steps
     if not args.no_e2e:
         xh = {k: v.cpu().pin_memory() for k, v in x.items()}
         oh = torch.empty((B, L, H, d), dtype=dt).pin_memory()
@@ -348,14 +428,14 @@ def run_gpu(args):
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(args.e2e_steps):
+        for _ in range(e2e_steps):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
         tensor_bytes = B * L * H * d * x["q"].element_size()
-        e2e = {"value": job_throughput(world, flops, args.e2e_steps, e2e_ms), "unit": "TFLOP/s",
-               "ms_per_step": e2e_ms / args.e2e_steps,
+        e2e = {"value": job_throughput(world, flops, e2e_steps, e2e_ms), "unit": "TFLOP/s",
+               "ms_per_step": e2e_ms / e2e_steps, "steps": e2e_steps,
                "h2d_bytes_per_step": 6 * tensor_bytes,
                "d2h_bytes_per_step": 2 * tensor_bytes + B * H * L * 4}
         del xh, oh, toh, lseh, staging
@@ -377,19 +457,16 @@ def run_gpu(args):
                                                   FALLBACK_PEAKS["bf16_tflops_sustained"])),
                 "kernel": "attn_jvp_tc_kernel<128, true> (CTA pairs)" if d == 128 else "attn_jvp_tc_kernel<64, false>",
                 "flops_per_launch": flops, "avg_launch_ms": avg_launch_ms}
-    cpu = None
+    cpu, parity = None, None
     if world == 1 and not args.no_cpu_baseline:
-        v, rows, secs, threads = oracle_sample(w, budget_s=args.cpu_budget)
-        cpu = {"value": v / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-               "sample": (f"{rows} seeded random query rows of one head, {secs:.1f} s of float64 "
-                          f"oracle work; effective FLOPs = 12 d x admissible pairs of those rows")}
+        cpu, parity = oracle_check_and_time(w, x, (o, to, lse), budget_s=args.cpu_budget)
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "pct_of_peak": 100.0 * value / world / peak,
             "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
             "config": workload_config(w, world), "roofline": roofline, "cpu_baseline": cpu,
-            "e2e": e2e, "gpu_launches": args.steps, "clocks": clk}
+            "e2e": e2e, "parity": parity, "gpu_launches": args.steps, "clocks": clk}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -569,7 +646,8 @@ def main():
     ap.add_argument("--workload", default="framewise_tf_bf16")
     ap.add_argument("--heads", type=int, default=None, help="override H (profiling a smaller case)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=None,
+                    help="timed steps of the end-to-end leg (default: --steps)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)

@@ -200,8 +200,10 @@ const char* attn_jvp_status_string(int status);
  * attn_jvp_fwd_noalloc - attn_jvp_fwd for callers that cannot allocate device
  * memory (an allocator-free runtime, a plugin host that owns every device
  * buffer, code running where cudaMalloc is forbidden or would break a memory
- * budget). It allocates nothing itself: not on the first call, not later.
- * There is no counterpart in the pages; it is an addition of this library.
+ * budget). It allocates no device memory: not on the first call, not later.
+ * (Its host-side work lists are built in fixed thread-local arrays, not on
+ * the heap.) There is no counterpart in the pages; it is an addition of this
+ * library.
  *
  * The bf16 kernel needs one word of scratch device memory besides its inputs
  * and outputs: the status word that a bounded wait sets when it runs out.
@@ -216,9 +218,10 @@ const char* attn_jvp_status_string(int status);
  *
  * Only bf16 is accepted (the fp32 kernel needs no scratch; use attn_jvp_fwd).
  * Arguments, layout and outputs are those of attn_jvp_fwd. Unlike it, this
- * call clears the scratch word on `stream`, launches, waits for `stream` and
- * returns the status of the launched work, so a bounded-wait timeout is
- * reported here as ATTN_JVP_ERR_DEVICE_TIMEOUT.
+ * call is synchronous: it clears the scratch word on `stream`, launches,
+ * copies the word back on `stream`, waits for `stream` and returns the
+ * status of the launched work, so a bounded-wait timeout is reported here as
+ * ATTN_JVP_ERR_DEVICE_TIMEOUT.
  *
  * The first call on a device (with that device current) looks up the array's
  * device address and the kernels' launch attributes; make that first call

@@ -5,5 +5,5 @@ import this package. It shares no code with the CUDA library.
 """
 from .attn_jvp_oracle import (  # noqa: F401
     BLOCK_CAUSAL, TEACHER_FORCING, allowed, attn_forward_dense, attn_jvp_dense,
-    attn_jvp_rows, count_pairs_bruteforce, effective_flops, mask_matrix, seq_len,
+    attn_jvp_rows, count_pairs_bruteforce, mask_matrix, seq_len,
 )

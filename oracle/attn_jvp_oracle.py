@@ -390,9 +390,3 @@ def rope_angles_1d(L: int, d: int, base: float = 10000.0) -> Tuple[np.ndarray, n
     t = np.arange(L, dtype=np.float64)[:, None]
     theta = base ** (-2.0 * np.arange(d // 2, dtype=np.float64) / d)[None, :]
     return np.cos(t * theta), np.sin(t * theta)
-
-
-def effective_flops(pairs: int, d: int) -> int:
-    """Algorithmic FLOPs of one call: 12 d per admissible pair (S: 2d,
-    tS: 4d, P V: 2d, tP V + P tV: 4d)."""
-    return 12 * d * pairs

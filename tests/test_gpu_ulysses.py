@@ -1,12 +1,15 @@
 """The Ulysses path on a GPU with the library's kernels as the local attention
 and backward (NCCL process group of one rank: the exchange is the identity,
 the kernels and the layout code are the real ones). Its outputs must equal a
-direct call's, bit for bit.
+direct call's, bit for bit, and the float64 oracle's within the parity
+tolerances. The exchange across several ranks, with these kernels inside it,
+is tested in test_gpu_ulysses_ranks.py.
 """
 import datetime
 import os
 import socket
 
+import numpy as np
 import pytest
 import torch
 import torch.distributed as dist
@@ -14,8 +17,16 @@ import torch.distributed as dist
 import attention_jvp_attn_b200 as aj
 from attention_jvp_attn_b200 import inputs as wl
 from attention_jvp_attn_b200.ulysses import ulysses_attn_jvp, ulysses_attn_jvp_bwd
+from oracle import attn_jvp_oracle as orc
 
 pytestmark = pytest.mark.gpu
+
+
+def _close(got, ref, tol):
+    g = got.double().cpu().numpy()
+    err = np.abs(g - ref) / (1.0 + np.abs(ref))
+    assert np.isfinite(g).all()
+    assert err.max() <= tol, f"max scaled error {err.max():.3e} > {tol}"
 
 
 def _free_port():
@@ -45,6 +56,9 @@ def test_ulysses_single_rank_equals_direct_call(cuda_device, nccl_group, d):
     assert aj.sync_status() == 0
     for u, v in zip(a, b):
         assert torch.equal(u.view(torch.uint8), v.contiguous().view(torch.uint8))
+    O, tO, LSE = orc.attn_jvp_dense(*(t.cpu() for t in ins), w.mode, w.chunk_tokens, w.n_chunks)
+    for got, ref, tol in zip(b, (O, tO, LSE), (2e-2, 2e-2, 1e-3)):
+        _close(got, ref, tol)
 
 
 @pytest.mark.parametrize("d", [64, 128])
@@ -63,3 +77,6 @@ def test_ulysses_backward_single_rank_equals_direct_call(cuda_device, nccl_group
     assert aj.sync_status() == 0
     for u, v2 in zip(a, b):
         assert torch.equal(u.view(torch.uint8), v2.contiguous().view(torch.uint8))
+    ref = orc.attn_vjp_dense(q.cpu(), k.cpu(), v.cpu(), do.cpu(), *m)
+    for got, r in zip(b, ref):
+        _close(got, r, 2e-2)

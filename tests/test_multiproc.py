@@ -95,3 +95,28 @@ def test_reference_arm_prints_one_contract_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["config"]["workload"] == "framewise_tf_bf16"
+    # ms_per_step is the measured time of one bounded sample (about --ref-budget
+    # seconds of oracle work), not an extrapolation to a full call
+    assert 400.0 <= d["ms_per_step"] < 60000.0
+    assert d["extrapolated_full_call_ms"] > d["ms_per_step"]
+
+
+def test_bench_parity_leg_passes_on_oracle_outputs_and_catches_a_wrong_row():
+    # the CPU-baseline leg compares the oracle on sampled rows with the timed
+    # call's outputs; here the "GPU outputs" are the oracle's own, rounded to bf16
+    sys.path.insert(0, ROOT)
+    import torch
+    import bench
+    from attention_jvp_attn_b200 import inputs as wl
+    from oracle import attn_jvp_oracle as orc
+    w = wl.Workload("bench_parity", B=2, H=3, d=64, n_chunks=3, chunk_tokens=100, seed=3)
+    x = wl.make_inputs(w)
+    O, tO, L = orc.attn_jvp_dense(*(x[n] for n in wl.TENSOR_ORDER), w.mode, w.chunk_tokens,
+                                  w.n_chunks)
+    outs = (torch.from_numpy(O).bfloat16(), torch.from_numpy(tO).bfloat16(),
+            torch.from_numpy(L).float())
+    cpu, par = bench.oracle_check_and_time(w, x, outs, budget_s=0.3)
+    assert par["pass"] and par["rows"] > 0 and cpu["kind"] == "oracle" and cpu["value"] > 0
+    outs[1][1, 0, 2, 3] += 1.0  # row 0 of the last (batch, head) slice is always sampled
+    _, par = bench.oracle_check_and_time(w, x, outs, budget_s=0.1)
+    assert not par["pass"] and par["max_err_over_bound_tO"] > 1.0

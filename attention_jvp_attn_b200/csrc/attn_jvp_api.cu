@@ -161,16 +161,7 @@ float softmax_scale(const attn_jvp_shape* s) {
 }
 
 bool encode_bf16_map(CUtensorMap* map, const void* base, const attn_jvp_shape* s, int box_rows) {
-  const cuuint64_t dims[4] = {cuuint64_t(s->d), cuuint64_t(s->H), cuuint64_t(s->L),
-                              cuuint64_t(s->B)};
-  const cuuint64_t strides[3] = {cuuint64_t(s->d) * 2, cuuint64_t(s->H * s->d) * 2,
-                                 cuuint64_t(s->L * s->H * s->d) * 2};
-  const cuuint32_t box[4] = {64, 1, cuuint32_t(box_rows), 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return ajvp::encode_bf16_rows_map(map, base, s->B, s->L, s->H, s->d, box_rows);
 }
 
 MaskSpec mask_spec(attn_jvp_mask m, int64_t L) {
@@ -433,6 +424,32 @@ int noalloc_state(NoAllocState** out) {
 
 
 }  // namespace
+
+namespace ajvp {
+
+int device_status_word(unsigned int** word) {
+  DeviceState* st = nullptr;
+  const int rc = device_state(&st);
+  if (rc != ATTN_JVP_OK) return rc;
+  *word = st->status;
+  return ATTN_JVP_OK;
+}
+
+bool encode_bf16_rows_map(CUtensorMap* map, const void* base, int64_t B, int64_t L, int64_t H,
+                          int64_t d, int box_rows) {
+  if (!g_encode) return false;
+  const cuuint64_t dims[4] = {cuuint64_t(d), cuuint64_t(H), cuuint64_t(L), cuuint64_t(B)};
+  const cuuint64_t strides[3] = {cuuint64_t(d) * 2, cuuint64_t(H * d) * 2,
+                                 cuuint64_t(L * H * d) * 2};
+  const cuuint32_t box[4] = {64, 1, cuuint32_t(box_rows), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace ajvp
 
 extern "C" {
 

@@ -1,5 +1,7 @@
 // attn_jvp_bwd.cu - backward (vector-Jacobian product) of the masked primal
 // attention on CUDA cores, and its C ABI (attn_jvp_bwd, attn_jvp_bwd_groups).
+// bf16 problems the tensor-core kernels take (attn_jvp_bwd_tc.cu) go there;
+// the kernels in this file serve fp32 and bf16 sequences too short for them.
 //
 // The fused forward returns LSE so that a backward pass can rebuild P without
 // a second softmax pass (Causal-rCM summary page, App. B, last item); the
@@ -29,6 +31,7 @@
 #include <mutex>
 
 #include "attn_jvp.h"
+#include "kernels.cuh"
 #include "mask_schedule.cuh"
 
 namespace ajvp_bwd {
@@ -356,7 +359,7 @@ int device_ready() {
   if (major != 10 || minor != 0) return ATTN_JVP_ERR_NO_DEVICE;  // built for sm_100a only
   if (prepare_one<64, float>() != cudaSuccess || prepare_one<128, float>() != cudaSuccess ||
       prepare_one<64, __nv_bfloat16>() != cudaSuccess ||
-      prepare_one<128, __nv_bfloat16>() != cudaSuccess) {
+      prepare_one<128, __nv_bfloat16>() != cudaSuccess || ajvp::bwd_tc_prepare() != cudaSuccess) {
     cudaGetLastError();
     return ATTN_JVP_ERR_CUDA;
   }
@@ -421,6 +424,27 @@ int run(const attn_jvp_shape* s, BwdParams& p, void* stream) {
   p.scale = s->scale > 0.f ? s->scale : 1.0f / std::sqrt(static_cast<float>(s->d));
   p.scale_log2 = p.scale * kLog2e;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (s->dtype == ATTN_JVP_BF16 && ajvp::bwd_tc_supported(s->B, s->L, s->H, s->d)) {
+    ajvp::BwdTcArgs a;
+    a.q = p.q;
+    a.k = p.k;
+    a.v = p.v;
+    a.o = p.o;
+    a.dout = p.dout;
+    a.lse = p.lse;
+    a.dlse = p.dlse;
+    a.dq = p.dq;
+    a.dk = p.dk;
+    a.dv = p.dv;
+    a.B = s->B;
+    a.L = s->L;
+    a.H = s->H;
+    a.d = s->d;
+    a.mask = p.mask;
+    a.mask.groups = p.mask.mode == ajvp::kModeGroups ? p.groups : nullptr;
+    a.scale = p.scale;
+    return ajvp::bwd_tc_launch(a, st);
+  }
   cudaError_t e;
   if (s->dtype == ATTN_JVP_BF16)
     e = s->d == 128 ? launch<128, __nv_bfloat16>(p, st) : launch<64, __nv_bfloat16>(p, st);

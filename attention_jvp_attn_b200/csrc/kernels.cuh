@@ -73,4 +73,27 @@ size_t simt_smem_bytes(int d);
 cudaError_t simt_prepare(int d);
 cudaError_t simt_launch(int d, const SimtParams& p, cudaStream_t stream);
 
+// ---- bf16 backward on tensor cores (attn_jvp_bwd_tc.cu) ----
+struct BwdTcArgs {
+  const void *q, *k, *v, *o, *dout;  // [B, L, H, d] bf16
+  const float *lse, *dlse;           // [B, H, L]; dlse may be null
+  void *dq, *dk, *dv;                // [B, L, H, d] bf16; dq also serves as scratch
+  int64_t B, L, H, d;
+  MaskSpec mask;  // kModeGroups: mask.groups points to a host table of mask.n_groups groups
+  float scale;
+};
+cudaError_t bwd_tc_prepare();  // sets the kernels' shared-memory limits (once per device)
+// True if the tensor-core backward runs this shape (else the CUDA-core kernels do).
+bool bwd_tc_supported(int64_t B, int64_t L, int64_t H, int64_t d);
+int bwd_tc_launch(const BwdTcArgs& a, cudaStream_t stream);  // ATTN_JVP_* status
+
+// ---- services of the C ABI layer for the other kernel files ----
+// The current device's status word (bit 0: a bounded wait ran out), set up
+// once per device; returns an ATTN_JVP_* status.
+int device_status_word(unsigned int** word);
+// 4-D tensor map over a dense [B, L, H, d] bf16 array: boxes of 64 columns x
+// `box_rows` rows of one (batch, head), 128-byte swizzle, zero fill out of range.
+bool encode_bf16_rows_map(CUtensorMap* map, const void* base, int64_t B, int64_t L, int64_t H,
+                          int64_t d, int box_rows);
+
 }  // namespace ajvp

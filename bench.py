@@ -235,7 +235,7 @@ def oracle_sample(w, budget_s: float, seed: int = 0):
         total_pairs += pairs
         rows_done += batch
         if total_t < budget_s / 4:
-            batch *= 2
+            batch = min(2 * batch, 4096)
     return 12 * w.d * total_pairs / total_t, rows_done, total_t, _oracle_threads()
 
 
@@ -286,7 +286,7 @@ def oracle_check_and_time(w, x, outs, budget_s: float, seed: int = 0):
     while total_t < budget_s:
         check(b, h, x64, sorted(set(rng.integers(0, w.L, size=batch).tolist())))
         if total_t < budget_s / 4:
-            batch *= 2
+            batch = min(2 * batch, 4096)
     cpu = {"value": 12 * w.d * total_pairs / total_t / 1e12, "unit": "TFLOP/s",
            "cores": _oracle_threads(), "kind": "oracle",
            "sample": (f"{n_rows} query rows of (batch, head) slices {slices} of the timed "
@@ -527,9 +527,12 @@ def run_backward(args) -> int:
     from the workload's Q, K, V, the forward's O and LSE and a seeded random
     cotangent dO. One JSON line: CUDA-event median over `--steps` calls after
     `--warmup`, inputs resident. Effective FLOPs count 10 d per admissible
-    pair (the products S, dP, dV, dK, dQ at 2 d each); the fp32 CUDA-core
-    kernels execute 7 d fused multiply-adds per pair (14 d FLOPs), against a
-    peak of 148 SMs x 128 fp32 lanes x 2 FLOPs x the sampled SM clock."""
+    pair (the products S, dP, dV, dK, dQ at 2 d each). For bf16 the call runs
+    on the tensor cores in three launches (row statistics, then dK/dV per key
+    block, then dQ per query block); S and dP are formed in both the dK/dV
+    and the dQ kernel, so 14 d FLOPs per pair execute. The roofline peak is
+    the measured bf16 dense burst. fp32 runs on CUDA cores against a peak of
+    148 SMs x 128 fp32 lanes x 2 FLOPs x the sampled SM clock."""
     import torch
     import attention_jvp_attn_b200 as aj
     from attention_jvp_attn_b200 import inputs as wl
@@ -564,21 +567,33 @@ def run_backward(args) -> int:
         torch.cuda.synchronize(dev)
         ms.append(e0.elapsed_time(e1))
     ck = clocks.stop()
+    if aj.sync_status(dev) != 0:
+        raise SystemExit("device status error")
     ms.sort()
     med = ms[len(ms) // 2]
     pairs_total = flops_per_step(w) // (12 * w.d)
     eff = 10 * w.d * pairs_total / (med * 1e-3) / 1e12
-    executed = 14 * w.d * pairs_total / (med * 1e-3) / 1e12
-    mhz = (ck or {}).get("sm_mhz") or 1965.0
-    alu_peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
+    if w.dtype == "bf16":
+        peaks, kind = load_peaks()
+        peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        executed = 14 * w.d * pairs_total / (med * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": eff, "peak": peak, "unit": "TFLOP/s",
+                "frac": eff / peak, "peak_source": f"{kind} bf16 dense burst",
+                "executed_tflops": executed, "executed_frac": executed / peak,
+                "note": "achieved counts 10 d per pair; 14 d execute (S, dP in both kernels)",
+                "kernels": ["bwd_prep_kernel", "bwd_dkdv_tc_kernel", "bwd_dq_tc_kernel"]}
+    else:
+        executed = 14 * w.d * pairs_total / (med * 1e-3) / 1e12
+        mhz = (ck or {}).get("sm_mhz") or 1965.0
+        alu_peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
+        roof = {"bound": "alu", "achieved": executed, "peak": alu_peak, "unit": "TFLOP/s",
+                "frac": executed / alu_peak,
+                "note": "fp32 FMA pipe; 14 d FLOPs executed per pair"}
     print(json.dumps({"mode": "backward", "workload": w.name, "dtype": w.dtype,
                       "B": w.B, "H": w.H, "L": w.L, "d": w.d, "steps": args.steps,
                       "warmup": args.warmup, "ms": med, "ms_min": ms[0], "ms_max": ms[-1],
                       "metric": "backward effective TFLOP/s (10 d per admissible pair)",
-                      "value": eff, "unit": "TFLOP/s",
-                      "roofline": {"bound": "alu", "achieved": executed, "peak": alu_peak,
-                                   "unit": "TFLOP/s", "frac": executed / alu_peak,
-                                   "note": "fp32 FMA pipe; 14 d FLOPs executed per pair"},
+                      "value": eff, "unit": "TFLOP/s", "roofline": roof,
                       "clocks": ck}), flush=True)
     return 0
 

@@ -265,16 +265,24 @@ int attn_jvp_fwd_noalloc(const attn_jvp_shape* shape,
  *   stream     cudaStream_t to launch on
  *
  * All pointers 16-byte aligned; outputs must not overlap inputs or each
- * other. Arithmetic is fp32 on CUDA cores for both dtypes; bf16 outputs are
- * rounded to nearest even. Two launches (dQ per block of 32 query rows, dK
- * and dV per block of 32 keys): each output element has one writer, so
- * results are the same bits on every run. Keys that no row may attend to get
- * zero gradients. lse must be the forward's (finite) LSE of these inputs.
+ * other. Each output element has one writer, so results are the same bits
+ * on every run. Keys that no row may attend to get zero gradients. lse must
+ * be the forward's (finite) LSE of these inputs.
+ *
+ * bf16 (when 8 * 128 ceil(L/128) <= 2 d L, i.e. L >= 8 for d = 64 and
+ * L >= 4 for d = 128): tensor cores, fp32 accumulation, P and dS rounded to
+ * bf16 before the dV, dK and dQ products, outputs rounded to nearest even.
+ * Three launches: per-row D_i = dO_i . O_i - dLSE_i and LSE_i log2(e) (fp32,
+ * written into the dq buffer, which serves as scratch until the last launch
+ * overwrites it with dQ), then dK and dV per block of 128 keys, then dQ per
+ * block of 128 query rows. Its waits are bounded: a wait that runs out is
+ * reported by attn_jvp_sync_status as ATTN_JVP_ERR_DEVICE_TIMEOUT.
+ * fp32 (and bf16 below those lengths): fp32 arithmetic on CUDA cores, two
+ * launches (dQ per block of 32 query rows, dK and dV per block of 32 keys).
  *
  * Returns ATTN_JVP_OK after enqueueing, or an error code with nothing
  * launched (argument errors are found on the host before any device call).
- * Does not synchronize; it has no bounded waits, so attn_jvp_sync_status
- * reports only stream errors for it.
+ * Does not synchronize.
  */
 int attn_jvp_bwd(const attn_jvp_shape* shape,
                  const void* q, const void* k, const void* v,

@@ -93,6 +93,13 @@ CASES = {  # dtype, d, mask ((mode, c, n) or a group table), scale, dLSE
     "kvcache_f32_d64": ("f32", 64, [(300, 0, 300, 300, 300), (470, 0, 300, 300, 470)], None,
                         True),
     "scaled_bf16_d64": ("bf16", 64, (TF, 33, 3), 0.05, False),
+    # bf16 below the tensor-core path's minimum length (L = 3): CUDA-core kernels
+    "short_bf16_d64": ("bf16", 64, (BC, 1, 3), None, True),
+    # tensor-core path: several 128-key blocks and query tiles, ragged tail,
+    # chunk edges inside tiles, group table with a gap inside a query block
+    "tf_c300_bf16_d64_dlse": ("bf16", 64, (TF, 300, 2), None, True),
+    "gapped_bf16_d128": ("bf16", 128, [(200, 0, 100, 300, 400), (400, 50, 250, 250, 400)], None,
+                         False),
 }
 
 

@@ -106,6 +106,8 @@ def load(path: str = None) -> ctypes.CDLL:
         lib.attn_jvp_rope.argtypes = [ctypes.POINTER(Shape), vp, vp, vp, vp, vp, vp, vp, vp,
                                       vp, vp, vp]
         lib.attn_jvp_rope.restype = ctypes.c_int
+        lib.attn_jvp_debug_wait.argtypes = [ctypes.c_int64, ctypes.c_int32]
+        lib.attn_jvp_debug_wait.restype = ctypes.c_int
         lib.attn_jvp_version.argtypes = []
         lib.attn_jvp_version.restype = ctypes.c_int32
         _lib = lib

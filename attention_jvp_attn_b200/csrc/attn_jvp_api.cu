@@ -263,6 +263,12 @@ bool fill_work_lists(const MaskSpec& ms, int bh_count, int n_qtiles, int bm, int
   return true;
 }
 
+// Test-only settings of the bf16 forward launches of this host thread (see
+// attn_jvp_debug_wait): the bounded-wait limit and a tile at which unit 0's
+// MMA issuer waits on a barrier that nothing completes.
+thread_local uint64_t t_wait_ns = 4000000000ull;
+thread_local int t_stall_tile = -1;
+
 int launch_bf16(DeviceState* st, const attn_jvp_shape* s, const void* q, const void* k,
                 const void* v, const void* tq, const void* tk, const void* tv, const MaskSpec& ms,
                 void* o, void* to, float* lse, cudaStream_t stream) {
@@ -293,6 +299,8 @@ int launch_bf16(DeviceState* st, const attn_jvp_shape* s, const void* q, const v
   const float sc = softmax_scale(s);
   p.scale = sc;
   p.scale_log2 = sc * 1.4426950408889634f;
+  p.wait_ns = t_wait_ns;
+  p.stall_tile = t_stall_tile;
   p.order_len = fill_order(ms, p.n_qtiles, bmu, p.order);
 #ifdef AJVP_TRACE
   p.trace = g_trace;
@@ -339,6 +347,49 @@ int launch_f32(const attn_jvp_shape* s, const void* q, const void* k, const void
 }
 
 int64_t round256(int64_t x) { return (x + 255) & ~int64_t(255); }
+
+// attn_jvp_fwd_host: heads in up to kHostChunks chunks, two staging slots.
+constexpr int64_t kHostChunks = 4;
+
+// Copy streams and events of attn_jvp_fwd_host, created once per device and
+// kept (like the status word): a call creates nothing.
+struct HostPipe {
+  std::mutex mu;  // one host-path call at a time per device (the call is synchronous)
+  bool ready = false;
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr, done = nullptr;
+  cudaEvent_t inp[2] = {nullptr, nullptr}, comp[2] = {nullptr, nullptr},
+              outp[2] = {nullptr, nullptr};
+};
+HostPipe g_pipe[kMaxDevices];
+
+int host_pipe(HostPipe** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return ATTN_JVP_ERR_NO_DEVICE;
+  }
+  std::lock_guard<std::mutex> lock(g_mu);
+  HostPipe& pp = g_pipe[dev];
+  if (!pp.ready) {
+    const unsigned ef = cudaEventDisableTiming;
+    bool ok = cudaStreamCreateWithFlags(&pp.in, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&pp.out, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&pp.start, ef) == cudaSuccess &&
+              cudaEventCreateWithFlags(&pp.done, ef) == cudaSuccess;
+    for (int i = 0; ok && i < 2; ++i)
+      ok = cudaEventCreateWithFlags(&pp.inp[i], ef) == cudaSuccess &&
+           cudaEventCreateWithFlags(&pp.comp[i], ef) == cudaSuccess &&
+           cudaEventCreateWithFlags(&pp.outp[i], ef) == cudaSuccess;
+    if (!ok) {
+      cudaGetLastError();
+      return ATTN_JVP_ERR_CUDA;
+    }
+    pp.ready = true;
+  }
+  *out = &pp;
+  return ATTN_JVP_OK;
+}
 
 // Pointer checks and the launch for either dtype (shape and mask validated).
 int run_checked(const attn_jvp_shape* shape, const void* q, const void* k, const void* v,
@@ -478,8 +529,11 @@ int64_t attn_jvp_host_staging_bytes(const attn_jvp_shape* shape) {
   if (!shape || shape->B < 1 || shape->L < 1 || shape->H < 1 || shape->d < 1) return 0;
   if (shape->dtype != ATTN_JVP_BF16 && shape->dtype != ATTN_JVP_F32) return 0;
   const int64_t esz = shape->dtype == ATTN_JVP_BF16 ? 2 : 4;
-  const int64_t t = shape->B * shape->L * shape->H * shape->d * esz;
-  return 8 * round256(t) + round256(shape->B * shape->H * shape->L * 4);
+  const int64_t n_chunks = shape->H >= kHostChunks ? kHostChunks : shape->H;
+  const int64_t hc = (shape->H + n_chunks - 1) / n_chunks;
+  const int64_t slot = 8 * round256(shape->B * shape->L * hc * shape->d * esz) +
+                       round256(shape->B * hc * shape->L * 4);
+  return (n_chunks > 1 ? 2 : 1) * slot;
 }
 
 int attn_jvp_fwd_host(const attn_jvp_shape* shape, const void* h_q, const void* h_k,
@@ -493,25 +547,76 @@ int attn_jvp_fwd_host(const attn_jvp_shape* shape, const void* h_q, const void* 
     if (!ptr) return ATTN_JVP_ERR_INVALID_ARGUMENT;
   if (!d_buf) return ATTN_JVP_ERR_INVALID_ARGUMENT;
   if (reinterpret_cast<uintptr_t>(d_buf) & 255u) return ATTN_JVP_ERR_MISALIGNED;
+  HostPipe* hpp = nullptr;
+  rc = host_pipe(&hpp);
+  if (rc != ATTN_JVP_OK) return rc;
+  HostPipe& pp = *hpp;
+  std::lock_guard<std::mutex> call_lock(pp.mu);
+  const int64_t B = shape->B, L = shape->L, H = shape->H, d = shape->d;
   const int64_t esz = shape->dtype == ATTN_JVP_BF16 ? 2 : 4;
-  const int64_t tb = shape->B * shape->L * shape->H * shape->d * esz;
-  const int64_t lb = shape->B * shape->H * shape->L * 4;
+  // Heads go in chunks of hc: H2D of chunk c+1 (copy stream) overlaps the
+  // kernel of chunk c (caller's stream) and the D2H of chunk c-1 (second copy
+  // stream), through two staging slots.
+  const int64_t n_chunks = H >= kHostChunks ? kHostChunks : H;
+  const int64_t hc_max = (H + n_chunks - 1) / n_chunks;
+  const int64_t t_slot = round256(B * L * hc_max * d * esz);  // one tensor of a chunk
+  const int64_t l_slot = round256(B * hc_max * L * 4);
+  const int64_t slot_bytes = 8 * t_slot + l_slot;
+  const int n_slots = n_chunks > 1 ? 2 : 1;
   char* base = static_cast<char*>(d_buf);
-  void* d[8];
-  for (int i = 0; i < 8; ++i) d[i] = base + i * round256(tb);
-  float* d_lse = reinterpret_cast<float*>(base + 8 * round256(tb));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const void* hin[6] = {h_q, h_k, h_v, h_tq, h_tk, h_tv};
-  for (int i = 0; i < 6; ++i)
-    if (cudaMemcpyAsync(d[i], hin[i], tb, cudaMemcpyHostToDevice, s) != cudaSuccess) {
-      cudaGetLastError();
-      return ATTN_JVP_ERR_CUDA;
-    }
-  rc = attn_jvp_fwd(shape, d[0], d[1], d[2], d[3], d[4], d[5], mask, d[6], d[7], d_lse, stream);
-  if (rc != ATTN_JVP_OK) return rc;
-  if (cudaMemcpyAsync(h_o, d[6], tb, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-      cudaMemcpyAsync(h_to, d[7], tb, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-      cudaMemcpyAsync(h_lse, d_lse, lb, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
+  void* hout[2] = {h_o, h_to};
+  const size_t row = static_cast<size_t>(H * d * esz);  // host row pitch (one token, all heads)
+  bool ok = true;
+  // The copy streams start after work already queued on the caller's stream.
+  ok = ok && cudaEventRecord(pp.start, s) == cudaSuccess;
+  ok = ok && cudaStreamWaitEvent(pp.in, pp.start, 0) == cudaSuccess;
+  ok = ok && cudaStreamWaitEvent(pp.out, pp.start, 0) == cudaSuccess;
+  for (int64_t c = 0; ok && c < n_chunks; ++c) {
+    const int64_t h0 = c * hc_max;
+    const int64_t hc = std::min(hc_max, H - h0);
+    if (hc <= 0) break;
+    const int sl = static_cast<int>(c % n_slots);
+    char* slot = base + sl * slot_bytes;
+    void* dt[8];
+    for (int i = 0; i < 8; ++i) dt[i] = slot + i * t_slot;
+    float* d_lse = reinterpret_cast<float*>(slot + 8 * t_slot);
+    const size_t width = static_cast<size_t>(hc * d * esz);
+    // inputs of chunk c into slot sl, once the kernel of chunk c - 2 has read them
+    if (c >= n_slots) ok = ok && cudaStreamWaitEvent(pp.in, pp.comp[sl], 0) == cudaSuccess;
+    for (int i = 0; ok && i < 6; ++i)
+      ok = cudaMemcpy2DAsync(dt[i], width, static_cast<const char*>(hin[i]) + h0 * d * esz, row,
+                             width, static_cast<size_t>(B * L), cudaMemcpyHostToDevice,
+                             pp.in) == cudaSuccess;
+    ok = ok && cudaEventRecord(pp.inp[sl], pp.in) == cudaSuccess;
+    // the kernel of chunk c, once its inputs are in and chunk c - 2's outputs are out
+    ok = ok && cudaStreamWaitEvent(s, pp.inp[sl], 0) == cudaSuccess;
+    if (c >= n_slots) ok = ok && cudaStreamWaitEvent(s, pp.outp[sl], 0) == cudaSuccess;
+    if (!ok) break;
+    attn_jvp_shape cs = *shape;
+    cs.H = hc;
+    rc = attn_jvp_fwd(&cs, dt[0], dt[1], dt[2], dt[3], dt[4], dt[5], mask, dt[6], dt[7], d_lse,
+                      stream);
+    if (rc != ATTN_JVP_OK) return rc;
+    ok = cudaEventRecord(pp.comp[sl], s) == cudaSuccess;
+    // outputs of chunk c to the host
+    ok = ok && cudaStreamWaitEvent(pp.out, pp.comp[sl], 0) == cudaSuccess;
+    for (int i = 0; ok && i < 2; ++i)
+      ok = cudaMemcpy2DAsync(static_cast<char*>(hout[i]) + h0 * d * esz, row, dt[6 + i], width,
+                             width, static_cast<size_t>(B * L), cudaMemcpyDeviceToHost,
+                             pp.out) == cudaSuccess;
+    // LSE: [B, hc, L] of the chunk into rows (b, h0 .. h0 + hc) of [B, H, L]
+    ok = ok && cudaMemcpy2DAsync(h_lse + h0 * L, static_cast<size_t>(H * L * 4), d_lse,
+                                 static_cast<size_t>(hc * L * 4), static_cast<size_t>(hc * L * 4),
+                                 static_cast<size_t>(B), cudaMemcpyDeviceToHost,
+                                 pp.out) == cudaSuccess;
+    ok = ok && cudaEventRecord(pp.outp[sl], pp.out) == cudaSuccess;
+  }
+  // The caller's stream ends after the last copy out.
+  ok = ok && cudaEventRecord(pp.done, pp.out) == cudaSuccess;
+  ok = ok && cudaStreamWaitEvent(s, pp.done, 0) == cudaSuccess;
+  if (!ok) {
     cudaGetLastError();
     return ATTN_JVP_ERR_CUDA;
   }
@@ -596,6 +701,14 @@ int32_t attn_jvp_schedule_tiles(attn_jvp_mask mask, int64_t L, int32_t block_m, 
 }
 
 int32_t attn_jvp_version(void) { return 100; }
+
+int attn_jvp_debug_wait(int64_t limit_ns, int32_t stall_tile) {
+  if (limit_ns < 0 || limit_ns > int64_t(60) * 1000000000) return ATTN_JVP_ERR_INVALID_ARGUMENT;
+  if (stall_tile < -1) return ATTN_JVP_ERR_INVALID_ARGUMENT;
+  t_wait_ns = limit_ns == 0 ? 4000000000ull : static_cast<uint64_t>(limit_ns);
+  t_stall_tile = stall_tile;
+  return ATTN_JVP_OK;
+}
 
 int attn_jvp_fwd_noalloc(const attn_jvp_shape* shape, const void* q, const void* k,
                          const void* v, const void* tq, const void* tk, const void* tv,

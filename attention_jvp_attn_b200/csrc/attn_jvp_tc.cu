@@ -101,8 +101,8 @@ struct TcCfg {
   static_assert(TILE == 16384, "16 KB tiles");
   static constexpr int DATA = 2 * QBYTES + NP * 2 * TILE;
   static constexpr int XCH = 2 * BM * 4 + 32;     // row statistics [2][BM] floats + flags [2][4]
-  static constexpr int NBAR = 2 * NP + 9 + 8;
-  static constexpr int BYTES = 1024 + DATA + XCH + NBAR * 8 + 16;
+  static constexpr int NBAR = 2 * NP + 9 + 8 + 2;  // + peer_done, stall
+  static constexpr int BYTES = 1024 + DATA + XCH + NBAR * 8 + 32;
   static constexpr int ARRIVALS = PAIR ? 16 : 8;  // softmax warps arriving on s_free, p_full, u_full
   static constexpr int HALF = BN / 2;             // key columns per softmax warpgroup
   static constexpr int DH = D / 2;                // output columns per softmax warpgroup
@@ -181,8 +181,11 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
   uint64_t* s_free = bars + 2 * C::NP + 8;
   uint64_t* xa = bars + 2 * C::NP + 9;   // [4] row-statistics exchange, first half
   uint64_t* xb = bars + 2 * C::NP + 13;  // [4] second half
+  uint64_t* peer_done = bars + 2 * C::NP + 17;  // pair: the peer's producer has published its counts
+  uint64_t* stall = bars + 2 * C::NP + 18;      // test-only wait that nothing completes
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint32_t* peer_cnt = tmem_slot + 2;  // pair, leader: the peer's ring and Q copy counts
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -209,10 +212,10 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
       mbar_arrive(bar);
   };
   auto bwait = [&](uint64_t* bar, uint32_t parity) -> bool {
-    return mbar_wait(bar, parity, abort_flag, p.status);
+    return mbar_wait(bar, parity, abort_flag, p.status, p.wait_ns);
   };
   auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
-    return warp_wait(bar, parity, abort_flag, p.status);
+    return warp_wait(bar, parity, abort_flag, p.status, p.wait_ns);
   };
 
   if (threadIdx.x == 0) {
@@ -228,6 +231,8 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
     mbar_init(u_full, C::ARRIVALS);
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
+    mbar_init(peer_done, 1);
+    mbar_init(stall, 1);
     mbar_init(s_free, C::ARRIVALS);
     for (int i = 0; i < 4; ++i) {
       mbar_init(&xa[i], 64);
@@ -338,20 +343,51 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
           }
         }
       }
-      if (!ok) {
-        if constexpr (PAIR) {
-          // Abort: the copies complete on the leader's barriers, so wait for
-          // them by time (they depend on nothing but memory) before exiting.
-          const uint64_t t0 = globaltimer_ns();
-          while (globaltimer_ns() - t0 < 2000000ull) __nanosleep(1000);
-        } else if (lane == 0) {
-          // Abort: let every copy already issued land before the CTA exits.
-          for (uint32_t s = 0; s < C::NP && s < ctr; ++s) {
-            const uint32_t last = ctr - 1 - ((ctr - 1 + C::NP - s) % C::NP);
-            mbar_wait_drain(&full[s], (last / C::NP) & 1, 200000000ull);
+      if constexpr (PAIR) {
+        // Both CTAs' copies complete on the leader's barriers, which only the
+        // leader arms. Before the CTAs can leave (the cluster barrier at the
+        // end), the leader makes every phase that either producer started
+        // complete: the peer publishes how many ring elements and Q tiles it
+        // issued; where the counts differ (an abort stopped one producer
+        // first) the leader takes the missing half off the pending bytes
+        // (complete_tx) or arms the peer's extra copies, then waits for the
+        // last phase of every slot. On a normal end every phase is complete
+        // already and this costs one round trip.
+        if (lane == 0) {
+          const uint32_t per_el = 2 * C::TILE, per_q = 2 * C::QBYTES;  // one CTA's bytes
+          if (rank != 0) {
+            st_cluster_u32(mapa_shared(smem_u32(peer_cnt), 0), ctr);
+            st_cluster_u32(mapa_shared(smem_u32(peer_cnt + 1), 0), q_issued);
+            mbar_arrive_remote_release(mapa_shared(smem_u32(peer_done), 0));
+          } else if (mbar_wait_acquire_cluster(peer_done, 0, p.wait_ns + 100000000ull)) {
+            const uint32_t c_peer = peer_cnt[0], q_peer = peer_cnt[1];
+            for (uint32_t e = min(ctr, c_peer); e < max(ctr, c_peer); ++e) {
+              if (e < ctr)
+                mbar_complete_tx(&full[e % C::NP], per_el);
+              else
+                mbar_arrive_expect_tx(&full[e % C::NP], per_el);
+            }
+            for (uint32_t i = min(q_issued, q_peer); i < max(q_issued, q_peer); ++i) {
+              if (i < q_issued)
+                mbar_complete_tx(q_full, per_q);
+              else
+                mbar_arrive_expect_tx(q_full, per_q);
+            }
+            const uint32_t n = max(ctr, c_peer), nq = max(q_issued, q_peer);
+            for (uint32_t s = 0; s < C::NP && s < n; ++s) {
+              const uint32_t last = n - 1 - ((n - 1 + C::NP - s) % C::NP);
+              mbar_wait_drain(&full[s], (last / C::NP) & 1, 200000000ull);
+            }
+            if (nq > 0) mbar_wait_drain(q_full, (nq - 1) & 1, 200000000ull);
           }
-          if (q_issued > 0) mbar_wait_drain(q_full, (q_issued - 1) & 1, 200000000ull);
         }
+      } else if (!ok && lane == 0) {
+        // Abort: let every copy already issued land before the CTA exits.
+        for (uint32_t s = 0; s < C::NP && s < ctr; ++s) {
+          const uint32_t last = ctr - 1 - ((ctr - 1 + C::NP - s) % C::NP);
+          mbar_wait_drain(&full[s], (last / C::NP) & 1, 200000000ull);
+        }
+        if (q_issued > 0) mbar_wait_drain(q_full, (q_issued - 1) & 1, 200000000ull);
       }
     }
     __syncwarp();
@@ -437,6 +473,9 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
           const uint32_t aK1 = el_addr(jk), aTK1 = aK1 + C::TILE;
           bool s_done = !has_next, rdy_p = false, rdy_v = false, rdy_u = false, rdy_k = false;
           AJVP_EV(g, 14);
+          // Test-only: the first unit waits at tile stall_tile on a barrier
+          // that nothing completes, so the wait runs out after wait_ns.
+          if (static_cast<int>(g) == p.stall_tile && cta == 0 && !wwait(stall, 0)) break;
           auto issue_s = [&](auto hook) {
             tc_fence_after();
             AJVP_EV(g, 12);
@@ -565,7 +604,7 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
             if (*abort_flag) { ok = 0; break; }
             const uint64_t now = globaltimer_ns();
             if (t0 == 0) t0 = now;
-            if (now - t0 > kWaitTimeoutNs) {
+            if (now - t0 > p.wait_ns) {
               *abort_flag = 1;
               atomicOr(p.status, kStatusTimeout);
               ok = 0;
@@ -586,11 +625,11 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
     auto exchange = [&](float mine, float& theirs) -> bool {
       *my_x = mine;
       mbar_arrive(&xa[sub]);
-      if (!warp_wait(&xa[sub], xa_ph, abort_flag, p.status)) return false;
+      if (!warp_wait(&xa[sub], xa_ph, abort_flag, p.status, p.wait_ns)) return false;
       xa_ph ^= 1;
       theirs = *other_x;
       mbar_arrive(&xb[sub]);
-      if (!warp_wait(&xb[sub], xb_ph, abort_flag, p.status)) return false;
+      if (!warp_wait(&xb[sub], xb_ph, abort_flag, p.status, p.wait_ns)) return false;
       xb_ph ^= 1;
       return true;
     };

@@ -33,6 +33,8 @@ struct TcParams {
   // position b*H*n_qtiles + h*n_qtiles + qt; else unit u takes rounds of a snake over
   // positions, with the query block of position r within a head given by the order table
   int list_mode;
+  unsigned long long wait_ns;  // limit of every bounded wait (default 4 s)
+  int stall_tile;              // test only: >= 0 makes unit 0's MMA issuer wait at that tile
   uint16_t unit_start[kMaxUnits + 1];
 #ifdef AJVP_TRACE
   long long* trace;  // per-tile event clocks of one CTA (trace builds only)

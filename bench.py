@@ -471,6 +471,95 @@ def run_gpu(args):
     return 0
 
 
+def run_ulysses(args) -> int:
+    """Head-sharded (Ulysses) attention JVP over the process group: each rank
+    holds one sequence block [B, L/N, H, d] of the six inputs of the same
+    problem; an NCCL all-to-all turns them into full-sequence shards of H/N
+    heads, the kernel runs on them, and all-to-alls return O, tO and LSE to
+    sequence blocks. The whole problem is fixed as N grows ("strong"
+    scaling); value = the problem's effective FLOPs per step x steps / the
+    slowest rank's time. With one rank the exchange is the identity."""
+    import socket
+    import torch
+    import torch.distributed as dist
+    import attention_jvp_attn_b200 as aj
+    from attention_jvp_attn_b200 import inputs as wl
+    from attention_jvp_attn_b200.ulysses import ulysses_attn_jvp
+
+    rank = _env_int("RANK", 0)
+    world = _env_int("WORLD_SIZE", 1)
+    local = _env_int("LOCAL_RANK", 0)
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = workload_by_name(args.workload, args.heads)
+    if w.H % world or w.L % world:
+        raise SystemExit(f"--ulysses needs H ({w.H}) and L ({w.L}) divisible by {world} ranks")
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    else:
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0,
+                                world_size=1, timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    full = wl.make_inputs(w, device=dev)
+    Ls = w.L // world
+    x = [full[n][:, rank * Ls:(rank + 1) * Ls].contiguous() for n in wl.TENSOR_ORDER]
+    del full
+    torch.cuda.empty_cache()
+    mask = (w.mode, w.chunk_tokens, w.n_chunks)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        return ulysses_attn_jvp(*x, mask, w.scale)
+
+    for _ in range(max(args.warmup, 1)):
+        step()
+    st = aj.sync_status(dev)
+    if st != 0:
+        raise SystemExit(f"device status {st} after warm-up")
+    clocks = ClockSampler(local)
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.25)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    clk = clocks.stop()
+    st = aj.sync_status(dev)
+    if st != 0:
+        raise SystemExit(f"device status {st} after timed steps")
+    total_ms = max_over_ranks(t0.elapsed_time(t1), dev)
+    dist.barrier()
+    dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    flops = flops_per_step(w)
+    value = flops * args.steps / (total_ms * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    cfg = workload_config(w, world)
+    cfg["parallelism"] = f"Ulysses head sharding over {world} ranks (NCCL all-to-all)"
+    cfg["global_batch"] = w.B
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+            "pct_of_peak": 100.0 * value / world / peak,
+            "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": cfg, "mode": "ulysses", "gpu_launches": args.steps, "clocks": clk}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_sweep(args) -> int:
     """Sweep (config 5): every point of inputs.sweep_points() on one GPU, one
     JSON line each (CUDA-event median of `--steps` launches after `--warmup`),
@@ -673,6 +762,8 @@ def main():
                     help="time the backward of the primal attention on one GPU (one JSON line)")
     ap.add_argument("--rope", action="store_true",
                     help="time the rotary embedding of Q, K, tQ, tK on one GPU (one JSON line)")
+    ap.add_argument("--ulysses", action="store_true",
+                    help="one problem sharded over the ranks by heads (NCCL all-to-all; strong scaling)")
     args = ap.parse_args()
     if args.warmup < 0 or args.steps < 1:
         raise SystemExit("need --steps >= 1 and --warmup >= 0")
@@ -684,6 +775,8 @@ def main():
         return run_backward(args)
     if args.rope:
         return run_rope(args)
+    if args.ulysses:
+        return run_ulysses(args)
     return run_gpu(args)
 
 

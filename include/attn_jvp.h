@@ -164,7 +164,15 @@ int attn_jvp_fwd_groups(const attn_jvp_shape* shape,
  * attn_jvp_fwd_host - the same operation on HOST buffers: copies the six
  * inputs host->device, runs attn_jvp_fwd, copies O, tO and LSE device->host
  * and waits for the stream. Host buffers should be pinned (page-locked) for
- * the copies to run at full speed; pageable memory also works.
+ * the copies to run at full speed (and to overlap with the kernel); pageable
+ * memory also works.
+ *
+ * The heads go in up to 4 chunks through two staging slots: the copies in
+ * of chunk c+1 and the copies out of chunk c-1 run on two copy streams while
+ * the kernel of chunk c runs on `stream`, ordered by events. The copy
+ * streams and events are created on the first call on a device and kept
+ * (like the status word); calls on one device are serialised by a lock.
+ * Results are the same bits as attn_jvp_fwd on the same inputs.
  *
  *   h_q..h_tv  host inputs, [B, L, H, d]
  *   h_o, h_to  host outputs, [B, L, H, d];  h_lse host output [B, H, L]
@@ -182,7 +190,9 @@ int attn_jvp_fwd_host(const attn_jvp_shape* shape,
                       void* h_o, void* h_to, float* h_lse,
                       void* d_buf, void* stream);
 
-/* Bytes of device staging attn_jvp_fwd_host needs for `shape` (0 on a bad shape). */
+/* Bytes of device staging attn_jvp_fwd_host needs for `shape` (0 on a bad shape):
+ * two slots of one chunk of heads (8 tensors and the LSE of ceil(H / 4) heads,
+ * each piece rounded up to 256 bytes), or one slot of the whole problem when H = 1. */
 int64_t attn_jvp_host_staging_bytes(const attn_jvp_shape* shape);
 
 /*
@@ -370,6 +380,30 @@ int32_t attn_jvp_schedule_tiles(attn_jvp_mask mask, int64_t L, int32_t block_m,
 int32_t attn_jvp_schedule_tiles_groups(const attn_jvp_group* groups, int32_t n_groups, int64_t L,
                                        int32_t block_m, int32_t block_n, int32_t q_tile,
                                        int32_t* tiles, uint8_t* full, int32_t cap);
+
+/*
+ * attn_jvp_debug_wait - TEST ONLY: drives the bf16 forward kernels' bounded
+ * waits to run out without a device fault (a wait on a barrier that nothing
+ * completes), so that the timeout path can be tested. Not part of the
+ * operation (the pages have no counterpart); it exists for failure-detection
+ * tests.
+ *
+ *   limit_ns    limit of every bounded wait of the bf16 forward kernels
+ *               launched later from the calling host thread; 0 restores
+ *               the default of 4 s (at most 60 s)
+ *   stall_tile  -1: no stall. >= 0: in those launches the first work unit's
+ *               MMA issuer, at its stall_tile-th key tile, waits on a barrier
+ *               that nothing completes. The wait runs out after limit_ns, the
+ *               kernel drains the copies and MMAs in flight, frees its tensor
+ *               memory and returns; attn_jvp_sync_status (or
+ *               attn_jvp_fwd_noalloc itself) reports
+ *               ATTN_JVP_ERR_DEVICE_TIMEOUT and the outputs are invalid.
+ *
+ * The settings are per host thread and stay until changed; call
+ * attn_jvp_debug_wait(0, -1) to restore normal operation. Returns
+ * ATTN_JVP_ERR_INVALID_ARGUMENT for values out of range.
+ */
+int attn_jvp_debug_wait(int64_t limit_ns, int32_t stall_tile);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
 int32_t attn_jvp_version(void);

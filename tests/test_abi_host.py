@@ -157,8 +157,29 @@ def test_rejects_null_and_misaligned_pointers(lib):
         assert _call(lib, s, m, ptrs) == _abi.ERR_MISALIGNED
 
 
+def _round256(x):
+    return (x + 255) // 256 * 256
+
+
 def test_staging_bytes(lib):
-    s = _abi.Shape(2, 128, 3, 64, 0, 0.0)
-    per = 2 * 128 * 3 * 64 * 2
-    assert lib.attn_jvp_host_staging_bytes(ctypes.byref(s)) == 8 * per + 2 * 3 * 128 * 4
+    # heads go in up to 4 chunks through two staging slots, each holding the
+    # 8 tensors and the LSE of one chunk (256-byte aligned pieces)
+    s = _abi.Shape(2, 128, 3, 64, 0, 0.0)  # 3 chunks of 1 head
+    slot = 8 * _round256(2 * 128 * 1 * 64 * 2) + _round256(2 * 1 * 128 * 4)
+    assert lib.attn_jvp_host_staging_bytes(ctypes.byref(s)) == 2 * slot
+    s = _abi.Shape(1, 100, 12, 128, 1, 0.0)  # fp32, 4 chunks of 3 heads
+    slot = 8 * _round256(100 * 3 * 128 * 4) + _round256(3 * 100 * 4)
+    assert lib.attn_jvp_host_staging_bytes(ctypes.byref(s)) == 2 * slot
+    s = _abi.Shape(1, 100, 1, 64, 0, 0.0)  # one head: one slot of the whole problem
+    assert lib.attn_jvp_host_staging_bytes(ctypes.byref(s)) == \
+        8 * _round256(100 * 64 * 2) + _round256(100 * 4)
     assert lib.attn_jvp_host_staging_bytes(ctypes.byref(_abi.Shape(0, 1, 1, 64, 0, 0.0))) == 0
+
+
+def test_debug_wait_settings_are_checked(lib):
+    # test-only bounded-wait settings: checked on the host, restored at the end
+    assert lib.attn_jvp_debug_wait(-1, -1) == _abi.ERR_INVALID_ARGUMENT
+    assert lib.attn_jvp_debug_wait(0, -2) == _abi.ERR_INVALID_ARGUMENT
+    assert lib.attn_jvp_debug_wait(61 * 10**9, -1) == _abi.ERR_INVALID_ARGUMENT
+    assert lib.attn_jvp_debug_wait(2_000_000, 3) == _abi.OK
+    assert lib.attn_jvp_debug_wait(0, -1) == _abi.OK

@@ -170,15 +170,21 @@ def test_deterministic(cuda_device):
         assert torch.equal(u, v)
 
 
-def test_host_buffer_entry_point(cuda_device):
-    w = wl.Workload("host", B=2, H=2, d=128, n_chunks=3, chunk_tokens=70, mode=TF, seed=9)
+@pytest.mark.parametrize("H,d,dtype", [(2, 128, "bf16"), (5, 64, "bf16"), (12, 128, "bf16"),
+                                        (3, 64, "f32")])
+def test_host_buffer_entry_point(cuda_device, H, d, dtype):
+    # heads go in chunks through two staging slots (5 heads: chunks of 2, 2, 1);
+    # the result must be the device entry point's, bit for bit
+    w = wl.Workload("host", B=2, H=H, d=d, n_chunks=3, chunk_tokens=70, mode=TF, seed=9 + H,
+                    dtype=dtype)
     x = wl.make_inputs(w, device="cpu")
     xh = {k: v.pin_memory() for k, v in x.items()}
     B, L, H, d = w.B, w.L, w.H, w.d
-    out = (torch.empty((B, L, H, d), dtype=torch.bfloat16).pin_memory(),
-           torch.empty((B, L, H, d), dtype=torch.bfloat16).pin_memory(),
+    dt = x["q"].dtype
+    out = (torch.empty((B, L, H, d), dtype=dt).pin_memory(),
+           torch.empty((B, L, H, d), dtype=dt).pin_memory(),
            torch.empty((B, H, L), dtype=torch.float32).pin_memory())
-    staging = torch.empty(aj.host_staging_bytes(B, L, H, d, torch.bfloat16), dtype=torch.uint8,
+    staging = torch.empty(aj.host_staging_bytes(B, L, H, d, dt), dtype=torch.uint8,
                           device=cuda_device)
     aj.attn_jvp_host(xh["q"], xh["k"], xh["v"], xh["tq"], xh["tk"], xh["tv"], w.mode,
                      w.chunk_tokens, w.n_chunks, staging, out)

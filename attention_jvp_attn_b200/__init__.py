@@ -193,11 +193,38 @@ def rope(q, k, tq, tk, cos, sin, out=None):
 
 
 def attn_jvp_rope(q, k, v, tq, tk, tv, cos, sin, mode: int, chunk_tokens: int, n_chunks: int,
-                  scale: Optional[float] = None):
+                  scale: Optional[float] = None, return_rotated: bool = False, out=None,
+                  rotated=None):
     """The attention JVP with RoPE applied to the queries and keys (and their
-    tangents) first: one rotation pass, then attn_jvp on the rotated tensors."""
-    qr, kr, tqr, tkr = rope(q, k, tq, tk, cos, sin)
-    return attn_jvp(qr, kr, v, tqr, tkr, tv, mode, chunk_tokens, n_chunks, scale)
+    tangents) first, in one call (one kernel launch for bf16): returns
+    (o, to, lse), and also the rotated (q, k, tq, tk) with return_rotated.
+    `rotated` may give the four buffers for the rotated tensors (the inputs
+    themselves for an in-place rotation)."""
+    ts = (q, k, v, tq, tk, tv)
+    for t in ts:
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("inputs must be contiguous CUDA tensors")
+        if t.shape != q.shape or t.dtype != q.dtype or t.device != q.device:
+            raise ValueError("q, k, v, tq, tk, tv must share shape, dtype and device")
+    B, L, H, d = q.shape
+    for t in (cos, sin):
+        if t.shape != (L, d // 2) or t.dtype != torch.float32 or t.device != q.device \
+                or not t.is_contiguous():
+            raise ValueError("cos and sin must be contiguous fp32 [L, d/2] on the inputs' device")
+    shape = _shape(q, scale)
+    rot = rotated if rotated is not None else tuple(torch.empty_like(q) for _ in range(4))
+    if out is None:
+        out = (torch.empty_like(q), torch.empty_like(q),
+               torch.empty((B, H, L), dtype=torch.float32, device=q.device))
+    lib = _abi.load()
+    with torch.cuda.device(q.device):
+        rc = lib.attn_jvp_fwd_rope(ctypes.byref(shape), *(t.data_ptr() for t in ts),
+                                   cos.data_ptr(), sin.data_ptr(),
+                                   _mask(mode, chunk_tokens, n_chunks),
+                                   *(t.data_ptr() for t in rot), *(t.data_ptr() for t in out),
+                                   _stream_handle(q.device))
+    _abi.check(rc, "attn_jvp_fwd_rope")
+    return (tuple(out), tuple(rot)) if return_rotated else tuple(out)
 
 
 def host_staging_bytes(B: int, L: int, H: int, d: int, dtype: torch.dtype) -> int:

@@ -59,7 +59,7 @@ def load(path: str = None) -> ctypes.CDLL:
     with _lock:
         if _lib is not None and path is None:
             return _lib
-        path = path or os.environ.get("ATTN_JVP_LIB", LIB_PATH)
+        path = path or os.environ.get("ATTN_JVP_LIB") or LIB_PATH
         if not os.path.exists(path):
             raise RuntimeError(
                 f"CUDA library not built: {path} is missing "
@@ -106,6 +106,9 @@ def load(path: str = None) -> ctypes.CDLL:
         lib.attn_jvp_rope.argtypes = [ctypes.POINTER(Shape), vp, vp, vp, vp, vp, vp, vp, vp,
                                       vp, vp, vp]
         lib.attn_jvp_rope.restype = ctypes.c_int
+        lib.attn_jvp_fwd_rope.argtypes = [ctypes.POINTER(Shape), vp, vp, vp, vp, vp, vp, vp, vp,
+                                          Mask, vp, vp, vp, vp, vp, vp, vp, vp]
+        lib.attn_jvp_fwd_rope.restype = ctypes.c_int
         lib.attn_jvp_debug_wait.argtypes = [ctypes.c_int64, ctypes.c_int32]
         lib.attn_jvp_debug_wait.restype = ctypes.c_int
         lib.attn_jvp_version.argtypes = []

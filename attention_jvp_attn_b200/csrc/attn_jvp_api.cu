@@ -20,6 +20,8 @@ using ajvp::MaskSpec;
 
 constexpr int kMaxDevices = 64;
 constexpr int64_t kMaxSeq = int64_t(1) << 30;
+constexpr int kGridSlots = 1024;  // launches with a grid barrier in flight at once, at most
+constexpr size_t kStateBytes = 256 + kGridSlots * sizeof(unsigned long long);
 
 struct DeviceState {
   bool ready = false;
@@ -27,6 +29,11 @@ struct DeviceState {
   int sm_count = 0;
   int pair_clusters = 0;           // CTA pairs resident at once (0: pair kernel unavailable)
   unsigned int* status = nullptr;  // device status word (bit 0: a bounded wait ran out)
+  // Grid-barrier words of the fused rotary-embedding launches (kGridSlots of
+  // them after the status word, in the same allocation), and the launch count
+  // that tags them.
+  unsigned long long* grid_slots = nullptr;
+  unsigned int grid_epoch = 0;
 };
 
 std::mutex g_mu;
@@ -72,12 +79,13 @@ int device_state(DeviceState** out) {
       }
       g_encode = reinterpret_cast<EncodeTiledFn>(fn);
     }
-    if (cudaMalloc(&st.status, sizeof(unsigned int)) != cudaSuccess) {
+    if (cudaMalloc(&st.status, kStateBytes) != cudaSuccess) {
       cudaGetLastError();
       st.status = nullptr;
       return ATTN_JVP_ERR_CUDA;
     }
-    if (cudaMemset(st.status, 0, sizeof(unsigned int)) != cudaSuccess ||
+    st.grid_slots = reinterpret_cast<unsigned long long*>(reinterpret_cast<char*>(st.status) + 256);
+    if (cudaMemset(st.status, 0, kStateBytes) != cudaSuccess ||
         ajvp::tc_prepare(128) != cudaSuccess || ajvp::tc_prepare(64) != cudaSuccess ||
         ajvp::simt_prepare(128) != cudaSuccess || ajvp::simt_prepare(64) != cudaSuccess) {
       cudaGetLastError();
@@ -269,11 +277,39 @@ bool fill_work_lists(const MaskSpec& ms, int bh_count, int n_qtiles, int bm, int
 thread_local uint64_t t_wait_ns = 4000000000ull;
 thread_local int t_stall_tile = -1;
 
+// Rotary embedding in the same launch: q, k, tq, tk are rotated into the
+// four `out` buffers (which the attention then reads) by the cos/sin tables.
+struct RopeArgs {
+  const float* cos;
+  const float* sin;
+  void* out[4];
+};
+
 int launch_bf16(DeviceState* st, const attn_jvp_shape* s, const void* q, const void* k,
                 const void* v, const void* tq, const void* tk, const void* tv, const MaskSpec& ms,
-                void* o, void* to, float* lse, cudaStream_t stream) {
+                void* o, void* to, float* lse, cudaStream_t stream,
+                const RopeArgs* rope = nullptr) {
   static thread_local ajvp::TcParams p;  // large (order table): not on the stack
   std::memset(&p, 0, offsetof(ajvp::TcParams, order));
+  if (rope) {
+    const void* src[4] = {q, k, tq, tk};
+    for (int i = 0; i < 4; ++i) {
+      p.rope_src[i] = src[i];
+      p.rope_dst[i] = rope->out[i];
+    }
+    p.rope = 1;
+    p.rope_cos = rope->cos;
+    p.rope_sin = rope->sin;
+    {
+      std::lock_guard<std::mutex> lock(g_mu);
+      p.grid_epoch = st->grid_epoch++;
+    }
+    p.grid_slot = st->grid_slots + (p.grid_epoch % kGridSlots);
+    q = rope->out[0];
+    k = rope->out[1];
+    tq = rope->out[2];
+    tk = rope->out[3];
+  }
   // d = 128 runs on CTA pairs: each CTA loads 64 of the 128 keys of a K or tK tile.
   const bool pair = s->d == 128;
   if (pair && st->pair_clusters <= 0) return ATTN_JVP_ERR_CUDA;
@@ -510,6 +546,33 @@ int attn_jvp_fwd(const attn_jvp_shape* shape, const void* q, const void* k, cons
   const int rc = validate(shape, mask);
   if (rc != ATTN_JVP_OK) return rc;
   return run_checked(shape, q, k, v, tq, tk, tv, mask_spec(mask, shape->L), o, to, lse, stream);
+}
+
+int attn_jvp_fwd_rope(const attn_jvp_shape* shape, const void* q, const void* k, const void* v,
+                      const void* tq, const void* tk, const void* tv, const float* cos,
+                      const float* sin, attn_jvp_mask mask, void* q_rot, void* k_rot,
+                      void* tq_rot, void* tk_rot, void* o, void* to, float* lse, void* stream) {
+  const int rc = validate(shape, mask);
+  if (rc != ATTN_JVP_OK) return rc;
+  const void* ptrs[15] = {q, k, v, tq, tk, tv, cos, sin, q_rot, k_rot, tq_rot, tk_rot, o, to, lse};
+  for (const void* ptr : ptrs)
+    if (!ptr) return ATTN_JVP_ERR_INVALID_ARGUMENT;
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return ATTN_JVP_ERR_MISALIGNED;
+  if (shape->B * shape->L * shape->H >= (int64_t(1) << 32)) return ATTN_JVP_ERR_UNSUPPORTED;
+  if (shape->dtype == ATTN_JVP_F32) {
+    // fp32: the stand-alone rotation pass, then the CUDA-core attention kernel
+    const int r = attn_jvp_rope(shape, q, k, tq, tk, cos, sin, q_rot, k_rot, tq_rot, tk_rot, stream);
+    if (r != ATTN_JVP_OK) return r;
+    return run_checked(shape, q_rot, k_rot, v, tq_rot, tk_rot, tv, mask_spec(mask, shape->L), o, to,
+                       lse, stream);
+  }
+  DeviceState* st = nullptr;
+  const int r = device_state(&st);
+  if (r != ATTN_JVP_OK) return r;
+  RopeArgs rope{cos, sin, {q_rot, k_rot, tq_rot, tk_rot}};
+  return launch_bf16(st, shape, q, k, v, tq, tk, tv, mask_spec(mask, shape->L), o, to, lse,
+                     static_cast<cudaStream_t>(stream), &rope);
 }
 
 int attn_jvp_fwd_groups(const attn_jvp_shape* shape, const void* q, const void* k, const void* v,

@@ -28,6 +28,7 @@
 #include <cstdint>
 
 #include "attn_jvp.h"
+#include "rope_math.cuh"
 
 namespace ajvp_rope {
 
@@ -106,11 +107,7 @@ __global__ void __launch_bounds__(kThreads) rope_kernel(const __grid_constant__ 
       s[i] = p.sin[a + i];
     }
 #pragma unroll
-    for (int i = 0; i < NP; ++i) {
-      const float x0 = x[2 * i], x1 = x[2 * i + 1];
-      x[2 * i] = x0 * c[i] - x1 * s[i];
-      x[2 * i + 1] = x0 * s[i] + x1 * c[i];
-    }
+    for (int i = 0; i < NP; ++i) ajvp::rope_rotate_pair(x[2 * i], x[2 * i + 1], c[i], s[i]);
     dst[v] = pack(x, T());
   }
 }

@@ -43,6 +43,7 @@
 
 #include "kernels.cuh"
 #include "ptx.cuh"
+#include "rope_math.cuh"
 #include "tiles.cuh"
 
 namespace ajvp {
@@ -156,6 +157,63 @@ __device__ __forceinline__ WorkItem decode_item(const TcParams& p, int pos) {
   return w;
 }
 
+// Rotation phase of the fused rotary embedding: one warp per (token, head)
+// row at a time, each lane 16 bytes (4 pairs) of one of q, k, tq, tk.
+template <int D>
+__device__ __forceinline__ void rope_phase(const TcParams& p) {
+  constexpr int VPR = D / 8;  // 16-byte vectors per row of one tensor
+  const unsigned rows = static_cast<unsigned>(p.B) * p.L * p.H;
+  const unsigned warps = gridDim.x * (blockDim.x >> 5);
+  const int lane = threadIdx.x & 31;
+  for (unsigned r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+    const unsigned t = (r / p.H) % p.L;  // token
+#pragma unroll
+    for (int j = lane; j < 4 * VPR; j += 32) {
+      const int which = j / VPR, col = (j % VPR) * 8;
+      const size_t off = static_cast<size_t>(r) * D + col;
+      const float4 c = *reinterpret_cast<const float4*>(p.rope_cos + static_cast<size_t>(t) * (D / 2) + col / 2);
+      const float4 sn = *reinterpret_cast<const float4*>(p.rope_sin + static_cast<size_t>(t) * (D / 2) + col / 2);
+      const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.rope_src[which]) + off);
+      float x[8] = {bf16lo_to_f32(u.x), bf16hi_to_f32(u.x), bf16lo_to_f32(u.y), bf16hi_to_f32(u.y),
+                    bf16lo_to_f32(u.z), bf16hi_to_f32(u.z), bf16lo_to_f32(u.w), bf16hi_to_f32(u.w)};
+      rope_rotate_pair(x[0], x[1], c.x, sn.x);
+      rope_rotate_pair(x[2], x[3], c.y, sn.y);
+      rope_rotate_pair(x[4], x[5], c.z, sn.z);
+      rope_rotate_pair(x[6], x[7], c.w, sn.w);
+      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.rope_dst[which]) + off) =
+          make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                     pack_bf16x2(x[6], x[7]));
+    }
+  }
+}
+
+// Grid barrier on a word shared by the launches that map to it: the high 32
+// bits tag the launch (epoch), the low 32 bits count its arrivals. The first
+// arrival of a launch retags the word. Bounded: false if the count did not
+// reach n within limit_ns. One thread per CTA calls it.
+__device__ __forceinline__ bool grid_sync(unsigned long long* slot, unsigned int epoch, unsigned int n,
+                                          uint64_t limit_ns) {
+  __threadfence();
+  const unsigned long long tag = static_cast<unsigned long long>(epoch) << 32;
+  const unsigned long long hi = ~0xffffffffull;
+  unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(slot);
+  while (true) {
+    const unsigned long long want = ((cur & hi) == tag) ? cur + 1 : (tag | 1ull);
+    const unsigned long long prev = atomicCAS(slot, cur, want);
+    if (prev == cur) break;
+    cur = prev;
+  }
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    const unsigned long long v = *reinterpret_cast<volatile unsigned long long*>(slot);
+    if ((v & hi) != tag || (v & 0xffffffffull) >= n) break;  // complete (or a later launch's)
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+    __nanosleep(256);
+  }
+  __threadfence();
+  return true;
+}
+
 template <int D, bool PAIR>
 __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_constant__ TcParams p) {
   using C = TcCfg<D, PAIR>;
@@ -218,6 +276,19 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
     return warp_wait(bar, parity, abort_flag, p.status, p.wait_ns);
   };
 
+  if (p.rope) {
+    // The rotated q, k, tq, tk first (every CTA a share), then all CTAs meet;
+    // the attention below reads them through TMA (the async proxy). A grid
+    // barrier that runs out reports a timeout; the kernel then still runs to
+    // its end, and its outputs are invalid.
+    rope_phase<D>(p);
+    fence_proxy_async_global();
+    __syncthreads();
+    if (threadIdx.x == 0 && !grid_sync(p.grid_slot, p.grid_epoch, gridDim.x, p.wait_ns))
+      atomicOr(p.status, kStatusTimeout);
+    __syncthreads();
+    fence_proxy_async_global();
+  }
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NP; ++i) {
       mbar_init(&full[i], 1);
@@ -658,6 +729,7 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
         tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
         tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
         tmem_wait_ld();
+        if (warp == 0 && lane == 0) AJVP_EVX(g, 10, __uint_as_float(sr[63]));
         if (!full_tile) {
           // admissible local columns of this row in this half tile, [s1, e1) U
           // [s2, e2), as 32-bit column masks
@@ -708,6 +780,7 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
         // by more than kRescaleTau): P first, the other half's maxima after.
         const bool spec = __all_sync(0xffffffffu, m_use != -INFINITY);
         if (spec) compute_p(m_use);
+        if (warp == 0 && lane == 0) AJVP_EVX(g, 11, ls3);
         // row maximum over both halves of the tile
         float their_max;
         if (!read_max(their_max)) { ok = false; break; }
@@ -769,6 +842,7 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
         uint32_t v[32];
         tmem_ld32(tTS, v);
         tmem_wait_ld();
+        if (warp == 0 && lane == 0) AJVP_EVX(g, 13, __uint_as_float(v[31]));
         tmem_st32(tTS, pk);
         tmem_wait_st();
         tc_fence_before();
@@ -918,14 +992,29 @@ int tc_pair_max_clusters(int sm_count) {
 }
 
 cudaError_t tc_launch(int d, const TcParams& p, int grid, cudaStream_t stream) {
+  // A launch with the rotation phase meets at a grid barrier: it asks for a
+  // cooperative launch, which fails rather than runs if its CTAs cannot all
+  // be resident at once.
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[2];
   if (d == 128) {
-    cudaLaunchConfig_t cfg;
-    cudaLaunchAttribute attr;
-    pair_config(&cfg, &attr, grid, stream);
-    return cudaLaunchKernelEx(&cfg, attn_jvp_tc_kernel<128, true>, p);
+    pair_config(&cfg, &attr[0], grid, stream);
+  } else {
+    cfg = cudaLaunchConfig_t{};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(kTcThreads, 1, 1);
+    cfg.dynamicSmemBytes = TcCfg<64, false>::BYTES;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 0;
   }
-  attn_jvp_tc_kernel<64, false><<<grid, kTcThreads, TcCfg<64, false>::BYTES, stream>>>(p);
-  return cudaGetLastError();
+  if (p.rope) {
+    attr[cfg.numAttrs].id = cudaLaunchAttributeCooperative;
+    attr[cfg.numAttrs].val.cooperative = 1;
+    cfg.numAttrs += 1;
+  }
+  if (d == 128) return cudaLaunchKernelEx(&cfg, attn_jvp_tc_kernel<128, true>, p);
+  return cudaLaunchKernelEx(&cfg, attn_jvp_tc_kernel<64, false>, p);
 }
 
 }  // namespace ajvp

@@ -33,6 +33,17 @@ struct TcParams {
   // position b*H*n_qtiles + h*n_qtiles + qt; else unit u takes rounds of a snake over
   // positions, with the query block of position r within a head given by the order table
   int list_mode;
+  // Rotary embedding in the same launch (rope != 0): every CTA first rotates
+  // a share of rope_src (q, k, tq, tk) into rope_dst, whose tensor maps the
+  // attention then reads; the CTAs meet at a grid barrier in between, on the
+  // word grid_slot tagged with grid_epoch.
+  int rope;
+  const void* rope_src[4];
+  void* rope_dst[4];
+  const float* rope_cos;  // [L, d/2]
+  const float* rope_sin;
+  unsigned long long* grid_slot;
+  unsigned int grid_epoch;
   unsigned long long wait_ns;  // limit of every bounded wait (default 4 s)
   int stall_tile;              // test only: >= 0 makes unit 0's MMA issuer wait at that tile
   uint16_t unit_start[kMaxUnits + 1];

@@ -11,6 +11,9 @@ scaling, no collective on the data path); rank 0 prints one JSON line.
 
 --impl reference times the float64 CPU oracle on the host cores instead (a
 bounded sample of the same workload per step) and prints the same line.
+Other modes, one JSON line each: --sweep (every sweep point), --backward (the
+backward of the primal attention), --rope (the rotary embedding pass),
+--ulysses (one problem sharded by heads over the ranks, strong scaling).
 """
 from __future__ import annotations
 
@@ -688,11 +691,16 @@ def run_backward(args) -> int:
 
 
 def run_rope(args) -> int:
-    """Rotary embedding of Q, K, tQ, tK (attn_jvp_rope) on one GPU: one JSON
-    line with the CUDA-event median over `--steps` calls after `--warmup`,
-    inputs resident (4 x the workload's tensor bytes, larger than L2). The
-    kernel is HBM-bound: algorithmic bytes are the four tensors read and
-    written plus the cos/sin tables read once."""
+    """Rotary embedding of Q, K, tQ, tK on one GPU, one JSON line.
+
+    - The stand-alone pass (attn_jvp_rope in C, `rope` in Python): HBM-bound;
+      algorithmic bytes are the four tensors read and written plus the cos/sin
+      tables read once. Timed over `--rope-calls` back-to-back calls, so that the
+      timed region spans several clock samples.
+    - The fused call (attn_jvp_fwd_rope: rotation and attention in one launch
+      for bf16) against attn_jvp alone on the same inputs: the CUDA-event
+      median of `--steps` calls each, after `--warmup`.
+    Inputs are resident (each tensor larger than L2)."""
     import numpy as np
     import torch
     import attention_jvp_attn_b200 as aj
@@ -706,39 +714,74 @@ def run_rope(args) -> int:
     cos = torch.from_numpy(np.cos(phi).astype(np.float32)).to(dev)
     sin = torch.from_numpy(np.sin(phi).astype(np.float32)).to(dev)
     ins = (x["q"], x["k"], x["tq"], x["tk"])
-    out = tuple(torch.empty_like(t) for t in ins)
+    rot = tuple(torch.empty_like(t) for t in ins)
 
-    def step():
-        aj.rope(*ins, cos, sin, out=out)
+    def rope_step():
+        aj.rope(*ins, cos, sin, out=rot)
 
     for _ in range(max(args.warmup, 1)):
-        step()
+        rope_step()
     if aj.sync_status(dev) != 0:
         raise SystemExit("device status error")
     clocks = ClockSampler(0)
     clocks.start()
-    ms = []
-    for _ in range(args.steps):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        step()
-        e1.record()
-        torch.cuda.synchronize(dev)
-        ms.append(e0.elapsed_time(e1))
+    time.sleep(0.25)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.rope_calls):
+        rope_step()
+    e1.record()
+    torch.cuda.synchronize(dev)
     ck = clocks.stop()
-    ms.sort()
-    med = ms[len(ms) // 2]
+    if aj.sync_status(dev) != 0:
+        raise SystemExit("device status error")
+    ms = e0.elapsed_time(e1) / args.rope_calls
     tensor_bytes = ins[0].numel() * ins[0].element_size()
     alg = 8 * tensor_bytes + 2 * cos.numel() * 4
     peaks, kind = load_peaks()
-    gbs = alg / (med * 1e-3) / 1e9
+    gbs = alg / (ms * 1e-3) / 1e9
+
+    outs = (torch.empty_like(x["q"]), torch.empty_like(x["q"]),
+            torch.empty((w.B, w.H, w.L), dtype=torch.float32, device=dev))
+
+    def fused_step():
+        aj.attn_jvp_rope(x["q"], x["k"], x["v"], x["tq"], x["tk"], x["tv"], cos, sin, w.mode,
+                         w.chunk_tokens, w.n_chunks, w.scale, out=outs, rotated=rot)
+
+    def plain_step():
+        aj.attn_jvp(x["q"], x["k"], x["v"], x["tq"], x["tk"], x["tv"], w.mode, w.chunk_tokens,
+                    w.n_chunks, w.scale, out=outs)
+
+    def median_ms(fn):
+        for _ in range(max(args.warmup, 1)):
+            fn()
+        t = []
+        for _ in range(args.steps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize(dev)
+            t.append(a.elapsed_time(b))
+        t.sort()
+        return t[len(t) // 2]
+
+    clocks2 = ClockSampler(0)
+    clocks2.start()
+    fused_ms = median_ms(fused_step)
+    plain_ms = median_ms(plain_step)
+    ck2 = clocks2.stop()
+    if aj.sync_status(dev) != 0:
+        raise SystemExit("device status error")
     print(json.dumps({"mode": "rope", "workload": w.name, "dtype": w.dtype, "B": w.B, "H": w.H,
-                      "L": w.L, "d": w.d, "steps": args.steps, "warmup": args.warmup,
-                      "ms": med, "ms_min": ms[0], "ms_max": ms[-1],
+                      "L": w.L, "d": w.d, "calls": args.rope_calls, "ms": ms,
                       "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
                                    "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
                                    "algorithmic_bytes": alg, "peak_kind": kind},
-                      "clocks": ck}), flush=True)
+                      "clocks": ck,
+                      "fused": {"ms": fused_ms, "forward_alone_ms": plain_ms,
+                                "overhead_pct": 100.0 * (fused_ms - plain_ms) / plain_ms,
+                                "steps": args.steps, "clocks": ck2}}), flush=True)
     return 0
 
 
@@ -762,6 +805,8 @@ def main():
                     help="time the backward of the primal attention on one GPU (one JSON line)")
     ap.add_argument("--rope", action="store_true",
                     help="time the rotary embedding of Q, K, tQ, tK on one GPU (one JSON line)")
+    ap.add_argument("--rope-calls", type=int, default=400,
+                    help="calls of the stand-alone rotation timed back to back (--rope)")
     ap.add_argument("--ulysses", action="store_true",
                     help="one problem sharded over the ranks by heads (NCCL all-to-all; strong scaling)")
     args = ap.parse_args()

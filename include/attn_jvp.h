@@ -345,6 +345,45 @@ int attn_jvp_rope(const attn_jvp_shape* shape,
                   void* q_out, void* k_out, void* tq_out, void* tk_out,
                   void* stream);
 
+/*
+ * attn_jvp_fwd_rope - attn_jvp_fwd with the rotary position embedding of
+ * attn_jvp_rope applied to q, k and their tangents tq, tk first, in the same
+ * launch for bf16 (Causal-rCM summary page, section 3, "KV Cache": RoPE on
+ * queries and keys, the attention's neighbour in the layer-level JVP). The
+ * operation is attn_jvp_fwd(R q, R k, v, R tq, R tk, tv) with R the rotation
+ * by the cos/sin tables; the rotated tensors R q, R k, R tq, R tk are also
+ * returned (the backward of the attention and a post-RoPE key cache need them).
+ *
+ *   q..tv       device inputs, [B, L, H, d] of shape->dtype
+ *   cos, sin    device tables, [L, d/2] float (token t, pair i), as for attn_jvp_rope
+ *   mask        as for attn_jvp_fwd
+ *   q_rot..tk_rot  device outputs, [B, L, H, d]: the rotated q, k, tq, tk; each
+ *               may be its own input (in place) and must not overlap any other
+ *   o, to, lse  device outputs, as for attn_jvp_fwd
+ *   stream      cudaStream_t to launch on
+ *
+ * bf16: one kernel launch. Its CTAs first rotate a share of q, k, tq, tk
+ * each (one pass over HBM), meet at a bounded grid barrier and then run the
+ * attention on the rotated tensors. The launch is cooperative (all its CTAs
+ * resident at once, or it fails with ATTN_JVP_ERR_CUDA). The barrier uses
+ * one of 1024 per-device words, tagged by a per-device launch count, so up
+ * to 1024 such calls may be in flight on a device at once. fp32: the
+ * rotation pass and then the CUDA-core kernel (two launches).
+ *
+ * All pointers 16-byte aligned; B * L * H < 2^32 (else ATTN_JVP_ERR_UNSUPPORTED).
+ * Returns ATTN_JVP_OK after enqueueing, or an error code with nothing
+ * launched. Does not synchronize; a bounded wait that runs out (the grid
+ * barrier included) is reported by attn_jvp_sync_status.
+ */
+int attn_jvp_fwd_rope(const attn_jvp_shape* shape,
+                      const void* q, const void* k, const void* v,
+                      const void* tq, const void* tk, const void* tv,
+                      const float* cos, const float* sin,
+                      attn_jvp_mask mask,
+                      void* q_rot, void* k_rot, void* tq_rot, void* tk_rot,
+                      void* o, void* to, float* lse,
+                      void* stream);
+
 /* ---- host-side helpers (need no GPU) ---------------------------------- */
 
 /* Number of admissible (query, key) pairs per (batch, head):

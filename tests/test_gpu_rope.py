@@ -97,3 +97,51 @@ def test_rope_then_attention_against_oracle(cuda_device, dtype, d, mode, c, n):
         err = np.abs(g - ref)
         assert np.isfinite(g).all() and (err <= tol * (1.0 + np.abs(ref))).all(), \
             (name, float(err.max()))
+
+
+# ---- the rotation and the attention in one call -------------------------------------------
+# attn_jvp_rope runs the rotation phase and the attention in one kernel launch
+# for bf16 (the CTAs meet at a grid barrier in between). Both halves compute
+# exactly what the separate rotation pass and attn_jvp compute, so the fused
+# call must give the same bits: the four rotated tensors, O, tO and LSE.
+
+@pytest.mark.parametrize("dtype,d,mode,c,n,B", [
+    ("bf16", 128, TF, 150, 3, 1),   # CTA pairs, ragged last 256-row block
+    ("bf16", 64, TF, 100, 4, 2),    # single CTAs, B = 2
+    ("bf16", 128, BC, 1560, 2, 1),  # longer chunks
+    ("bf16", 64, BC, 7, 5, 1),      # chunks shorter than a tile, L = 35
+    ("f32", 64, TF, 40, 2, 1),      # fp32: rotation pass, then the CUDA-core kernel
+])
+def test_fused_rope_equals_rotation_then_attention(cuda_device, dtype, d, mode, c, n, B):
+    L = orc.seq_len(mode, c, n)
+    H = 3
+    q, k, v, tq, tk, tv = _tensors(B, L, H, d, dtype, 70 + L + d, cuda_device, n=6)
+    cs, sn = _angles(L, d, "random", L + d)
+    cd, sd = torch.from_numpy(cs).to(cuda_device), torch.from_numpy(sn).to(cuda_device)
+    (o, to, lse), rot = aj.attn_jvp_rope(q, k, v, tq, tk, tv, cd, sd, mode, c, n,
+                                         return_rotated=True)
+    assert aj.sync_status() == 0
+    ref_rot = aj.rope(q, k, tq, tk, cd, sd)
+    ref = aj.attn_jvp(ref_rot[0], ref_rot[1], v, ref_rot[2], ref_rot[3], tv, mode, c, n)
+    assert aj.sync_status() == 0
+    for got, want in zip(rot + (o, to, lse), tuple(ref_rot) + tuple(ref)):
+        assert torch.equal(got.view(torch.uint8), want.view(torch.uint8))
+
+
+def test_fused_rope_in_place_and_repeated(cuda_device):
+    # rotated buffers = the inputs (in place); the next call, on the rotated
+    # tensors' originals again, uses the next grid-barrier word
+    B, L, H, d, mode, c, n = 1, 600, 2, 128, TF, 100, 3
+    q, k, v, tq, tk, tv = _tensors(B, L, H, d, "bf16", 5, cuda_device, n=6)
+    cs, sn = _angles(L, d, "random", 9)
+    cd, sd = torch.from_numpy(cs).to(cuda_device), torch.from_numpy(sn).to(cuda_device)
+    first = aj.attn_jvp_rope(q, k, v, tq, tk, tv, cd, sd, mode, c, n)
+    ins = [t.clone() for t in (q, k, tq, tk)]
+    second = aj.attn_jvp_rope(ins[0], ins[1], v, ins[2], ins[3], tv, cd, sd, mode, c, n,
+                              rotated=tuple(ins))
+    assert aj.sync_status() == 0
+    ref_rot = aj.rope(q, k, tq, tk, cd, sd)
+    for a, b in zip(first, second):
+        assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
+    for got, want in zip(ins, ref_rot):
+        assert torch.equal(got.view(torch.uint8), want.view(torch.uint8))

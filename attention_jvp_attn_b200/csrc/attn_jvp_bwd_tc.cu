@@ -407,14 +407,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_tc_kernel(const __gri
         }
       }
       // P^T = 2^(S^T s log2 e - LSE_i log2 e): 0 where masked or past L
+      // scalings on pairs of floats (FFMA2); S^T s log2 e - LSE_i log2 e
       uint32_t pk[32];
+      const float2 sc2 = make_float2(sl2, sl2);
 #pragma unroll
       for (int j = 0; j < 64; j += 4) {
         const float4 l4 = *reinterpret_cast<const float4*>(lse2 + j);
-        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[j]), sl2, -l4.x));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(sr[j + 1]), sl2, -l4.y));
-        const float p2 = ex2_approx(fmaf(__uint_as_float(sr[j + 2]), sl2, -l4.z));
-        const float p3 = ex2_approx(fmaf(__uint_as_float(sr[j + 3]), sl2, -l4.w));
+        const float2 x01 = __ffma2_rn(make_float2(__uint_as_float(sr[j]), __uint_as_float(sr[j + 1])),
+                                      sc2, make_float2(-l4.x, -l4.y));
+        const float2 x23 = __ffma2_rn(make_float2(__uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3])),
+                                      sc2, make_float2(-l4.z, -l4.w));
+        const float p0 = ex2_approx(x01.x), p1 = ex2_approx(x01.y);
+        const float p2 = ex2_approx(x23.x), p3 = ex2_approx(x23.y);
         sr[j] = __float_as_uint(p0);
         sr[j + 1] = __float_as_uint(p1);
         sr[j + 2] = __float_as_uint(p2);
@@ -433,21 +437,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_tc_kernel(const __gri
       uint32_t v[32];
       tmem_ld32(tDP, v);
       tmem_wait_ld();
+      // dS^T = P^T (dP^T - D_i) on pairs of floats (FADD2, FMUL2)
+      auto ds_pair = [&](int c, uint32_t v0, uint32_t v1, float2 d2) -> uint32_t {
+        const float2 ds = __fmul2_rn(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])),
+                                     __fadd2_rn(make_float2(__uint_as_float(v0), __uint_as_float(v1)),
+                                                make_float2(-d2.x, -d2.y)));
+        return pack_bf16x2(ds.x, ds.y);
+      };
 #pragma unroll
-      for (int j = 0; j < 32; j += 2) {
-        const float2 d2 = *reinterpret_cast<const float2*>(dd + j);
-        pk[j / 2] = pack_bf16x2(__uint_as_float(sr[j]) * (__uint_as_float(v[j]) - d2.x),
-                                __uint_as_float(sr[j + 1]) * (__uint_as_float(v[j + 1]) - d2.y));
-      }
+      for (int j = 0; j < 32; j += 2)
+        pk[j / 2] = ds_pair(j, v[j], v[j + 1], *reinterpret_cast<const float2*>(dd + j));
       tmem_ld32(tDP + 32, v);
       tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 32; j += 2) {
-        const float2 d2 = *reinterpret_cast<const float2*>(dd + 32 + j);
-        pk[16 + j / 2] =
-            pack_bf16x2(__uint_as_float(sr[32 + j]) * (__uint_as_float(v[j]) - d2.x),
-                        __uint_as_float(sr[33 + j]) * (__uint_as_float(v[j + 1]) - d2.y));
-      }
+      for (int j = 0; j < 32; j += 2)
+        pk[16 + j / 2] = ds_pair(32 + j, v[j], v[j + 1], *reinterpret_cast<const float2*>(dd + 32 + j));
       tmem_st32(tDP, pk);
       tmem_wait_st();
       tc_fence_before();
@@ -501,8 +505,13 @@ template <int D>
 struct DqCfg {
   static constexpr int CH = D / 64;
   static constexpr int TILE = kBB * D * 2;
-  static constexpr int NP = D == 128 ? 5 : 8;         // ring elements: K_j or V_j, one tile each
-  static constexpr int DATA = 2 * TILE + NP * TILE;   // Q, dO resident, then the ring
+  // Two rings: K_j is read by S_j (early) and dQ_j (late), V_j only by dP_j
+  // (early), so each ring is released at its own pace and a V load need not
+  // wait for a K slot.
+  static constexpr int NK = D == 128 ? 3 : 4;         // K ring slots
+  static constexpr int NV = D == 128 ? 2 : 4;         // V ring slots
+  static constexpr int NP = NK + NV;
+  static constexpr int DATA = 2 * TILE + NP * TILE;   // Q, dO resident, then the rings
   static constexpr int XCH = 2 * kBB * 4;             // partial dO.O exchange [2][128]
   static constexpr int NBAR = 2 * NP + 9 + 4;
   static constexpr int BYTES = 1024 + DATA + XCH + NBAR * 8 + 16;
@@ -599,14 +608,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_tc_kernel(const __grid_
       }
     }
     __syncwarp();
-    uint32_t e = 0;
+    // ring slot of K_j: j % NK; of V_j: NK + j % NV
+    int k_issued = 0, v_issued = 0;
     bool ok = true;
     for (int idx = 0; ok && idx < cnt; ++idx) {
       const int kt = sch.tile(idx);
 #pragma unroll 1
-      for (int which = 0; which < 2; ++which, ++e) {
-        const uint32_t el = e % C::NP;
-        if (!wwait(&empty[el], ((e / C::NP) & 1) ^ 1)) { ok = false; break; }
+      for (int which = 0; which < 2; ++which) {
+        const int n = which == 0 ? C::NK : C::NV;
+        const uint32_t el = (which == 0 ? 0 : C::NK) + idx % n;
+        if (!wwait(&empty[el], ((idx / n) & 1) ^ 1)) { ok = false; break; }
         if (elect_one()) {
           mbar_arrive_expect_tx(&full[el], C::TILE);
           const CUtensorMap* map = which == 0 ? &p.map_k : &p.map_v;
@@ -616,14 +627,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_tc_kernel(const __grid_
                              kt * kBB, b, keep);
         }
         __syncwarp();
+        if (which == 0)
+          k_issued = idx + 1;
+        else
+          v_issued = idx + 1;
       }
     }
     if (!ok && lane == 0) {
+      // Abort: let every copy already issued land before the CTA exits.
       if (cnt > 0) mbar_wait_drain(q_full, 0, 200000000ull);
-      for (uint32_t s = 0; s < C::NP && s < e; ++s) {
-        const uint32_t last = e - 1 - ((e - 1 + C::NP - s) % C::NP);
-        mbar_wait_drain(&full[s], (last / C::NP) & 1, 200000000ull);
-      }
+      for (int j = k_issued - 1; j >= 0 && j >= k_issued - C::NK; --j)
+        mbar_wait_drain(&full[j % C::NK], (j / C::NK) & 1, 200000000ull);
+      for (int j = v_issued - 1; j >= 0 && j >= v_issued - C::NV; --j)
+        mbar_wait_drain(&full[C::NK + j % C::NV], (j / C::NV) & 1, 200000000ull);
     }
     __syncwarp();
   } else if (warp == 9) {
@@ -634,43 +650,46 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_tc_kernel(const __grid_
     const uint32_t idesc_s = idesc_bf16_f32(128, kBB, 0);
     const uint32_t idesc_v = idesc_bf16_f32(128, D, 1);
     const uint32_t aQ = smem_u32(sQ), aDO = smem_u32(sDO), aRing = smem_u32(sRing);
-    auto el_addr = [&](uint32_t e) { return aRing + (e % C::NP) * C::TILE; };
-    auto el_full = [&](uint32_t e) { return &full[e % C::NP]; };
-    auto el_ph = [&](uint32_t e) { return (e / C::NP) & 1; };
+    // K_j in slot j % NK, V_j in slot NK + j % NV
+    auto k_slot = [&](int j) { return static_cast<uint32_t>(j % C::NK); };
+    auto v_slot = [&](int j) { return static_cast<uint32_t>(C::NK + j % C::NV); };
+    auto k_ph = [&](int j) { return static_cast<uint32_t>((j / C::NK) & 1); };
+    auto v_ph = [&](int j) { return static_cast<uint32_t>((j / C::NV) & 1); };
+    auto el_addr = [&](uint32_t slot) { return aRing + slot * C::TILE; };
     auto tm_dp = [&](int j) { return tmem + ((j & 1) ? C::TM_DP1 : C::TM_DP0); };
     if (cnt > 0) {
-      bool ok = wwait(q_full, 0) && wwait(el_full(0), 0);
+      bool ok = wwait(q_full, 0) && wwait(&full[k_slot(0)], 0);
       if (ok) {
         tc_fence_after();
-        mma_scores<D, kBB, kBB, false>(tmem + C::TM_S, aQ, el_addr(0), idesc_s, false);
+        mma_scores<D, kBB, kBB, false>(tmem + C::TM_S, aQ, el_addr(k_slot(0)), idesc_s, false);
         umma_commit(s_full);
-        ok = wwait(el_full(1), 0);
+        ok = wwait(&full[v_slot(0)], 0);
       }
       if (ok) {
         tc_fence_after();
-        mma_scores<D, kBB, kBB, false>(tm_dp(0), aDO, el_addr(1), idesc_s, false);
+        mma_scores<D, kBB, kBB, false>(tm_dp(0), aDO, el_addr(v_slot(0)), idesc_s, false);
         umma_commit(&dp_full[0]);
-        umma_commit(&empty[1 % C::NP]);
+        umma_commit(&empty[v_slot(0)]);
       }
       for (int idx = 0; ok && idx < cnt; ++idx) {
         const uint32_t ph = idx & 1;
         if (idx + 1 < cnt) {
-          const uint32_t ek = 2 * (idx + 1), ev = ek + 1;
-          if (!wwait(s_free, ph) || !wwait(el_full(ek), el_ph(ek))) break;
+          const int j = idx + 1;
+          if (!wwait(s_free, ph) || !wwait(&full[k_slot(j)], k_ph(j))) break;
           tc_fence_after();
-          mma_scores<D, kBB, kBB, false>(tmem + C::TM_S, aQ, el_addr(ek), idesc_s, false);
+          mma_scores<D, kBB, kBB, false>(tmem + C::TM_S, aQ, el_addr(k_slot(j)), idesc_s, false);
           umma_commit(s_full);
-          if (!wwait(el_full(ev), el_ph(ev))) break;
+          if (!wwait(&full[v_slot(j)], v_ph(j))) break;
           tc_fence_after();
-          mma_scores<D, kBB, kBB, false>(tm_dp(idx + 1), aDO, el_addr(ev), idesc_s, false);
-          umma_commit(&dp_full[(idx + 1) & 1]);
-          umma_commit(&empty[ev % C::NP]);
+          mma_scores<D, kBB, kBB, false>(tm_dp(j), aDO, el_addr(v_slot(j)), idesc_s, false);
+          umma_commit(&dp_full[j & 1]);
+          umma_commit(&empty[v_slot(j)]);
         }
         if (!wwait(&ds_full[idx & 1], (idx >> 1) & 1)) break;
         tc_fence_after();
-        const uint32_t ek = 2 * idx;
-        mma_values_split<kBB, false>(tmem + C::TM_DQ, tm_dp(idx), el_addr(ek), idesc_v, idx > 0);
-        umma_commit(&empty[ek % C::NP]);
+        mma_values_split<kBB, false>(tmem + C::TM_DQ, tm_dp(idx), el_addr(k_slot(idx)), idesc_v,
+                                     idx > 0);
+        umma_commit(&empty[k_slot(idx)]);
         if (idx == cnt - 1) umma_commit(acc_full);
       }
     }
@@ -746,26 +765,35 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_tc_kernel(const __grid_
             if (!((m >> j) & 1u)) sr[32 * q + j] = __float_as_uint(-INFINITY);
         }
       }
+      {
+        const float2 sc2 = make_float2(sl2, sl2), nl2 = make_float2(-lse2, -lse2);
 #pragma unroll
-      for (int j = 0; j < 64; ++j)
-        sr[j] = __float_as_uint(ex2_approx(fmaf(__uint_as_float(sr[j]), sl2, -lse2)));
+        for (int j = 0; j < 64; j += 2) {
+          const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[j]), __uint_as_float(sr[j + 1])),
+                                      sc2, nl2);
+          sr[j] = __float_as_uint(ex2_approx(x.x));
+          sr[j + 1] = __float_as_uint(ex2_approx(x.y));
+        }
+      }
       if (!wwait(&dp_full[idx & 1], (idx >> 1) & 1)) { ok = false; break; }
       tc_fence_after();
       const uint32_t tDP = tmem + lane_off + ((idx & 1) ? C::TM_DP1 : C::TM_DP0) + 64 * wg;
       uint32_t v[32], pk[32];
       tmem_ld32(tDP, v);
       tmem_wait_ld();
+      // dS = P (dP - D_t) on pairs of floats (FADD2, FMUL2)
+      const float2 nd2 = make_float2(-d_row, -d_row);
+      auto ds_pair = [&](int c, uint32_t v0, uint32_t v1) -> uint32_t {
+        const float2 ds = __fmul2_rn(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])),
+                                     __fadd2_rn(make_float2(__uint_as_float(v0), __uint_as_float(v1)), nd2));
+        return pack_bf16x2(ds.x, ds.y);
+      };
 #pragma unroll
-      for (int j = 0; j < 32; j += 2)
-        pk[j / 2] = pack_bf16x2(__uint_as_float(sr[j]) * (__uint_as_float(v[j]) - d_row),
-                                __uint_as_float(sr[j + 1]) * (__uint_as_float(v[j + 1]) - d_row));
+      for (int j = 0; j < 32; j += 2) pk[j / 2] = ds_pair(j, v[j], v[j + 1]);
       tmem_ld32(tDP + 32, v);
       tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 32; j += 2)
-        pk[16 + j / 2] =
-            pack_bf16x2(__uint_as_float(sr[32 + j]) * (__uint_as_float(v[j]) - d_row),
-                        __uint_as_float(sr[33 + j]) * (__uint_as_float(v[j + 1]) - d_row));
+      for (int j = 0; j < 32; j += 2) pk[16 + j / 2] = ds_pair(32 + j, v[j], v[j + 1]);
       tmem_st32(tDP, pk);
       tmem_wait_st();
       tc_fence_before();

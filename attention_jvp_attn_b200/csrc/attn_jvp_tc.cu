@@ -746,41 +746,44 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
               if (!((m >> j) & 1u)) sr[32 * q + j] = __float_as_uint(-INFINITY);
           }
         }
+        // three-input max: two new values per instruction, four chains
         float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-        for (int j = 0; j < C::HALF; j += 4) {
-          mx0 = fmaxf(mx0, __uint_as_float(sr[j]));
-          mx1 = fmaxf(mx1, __uint_as_float(sr[j + 1]));
-          mx2 = fmaxf(mx2, __uint_as_float(sr[j + 2]));
-          mx3 = fmaxf(mx3, __uint_as_float(sr[j + 3]));
+        for (int j = 0; j < C::HALF; j += 8) {
+          mx0 = fmax3(mx0, __uint_as_float(sr[j]), __uint_as_float(sr[j + 1]));
+          mx1 = fmax3(mx1, __uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3]));
+          mx2 = fmax3(mx2, __uint_as_float(sr[j + 4]), __uint_as_float(sr[j + 5]));
+          mx3 = fmax3(mx3, __uint_as_float(sr[j + 6]), __uint_as_float(sr[j + 7]));
         }
-        const float my_max = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        const float my_max = fmaxf(fmax3(mx0, mx1, mx2), mx3);
         tc_fence_before();
         publish_max(my_max);
         // P of this half tile at the running max mb (bf16, packed) and its row sum.
+        // The scalings and the row sums run on pairs of floats (FFMA2, FADD2).
         uint32_t pk[C::HALF / 2];
-        float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
+        float2 ls01 = make_float2(0.f, 0.f), ls23 = make_float2(0.f, 0.f);
         auto compute_p = [&](float mb) {
-          ls0 = ls1 = ls2 = ls3 = 0.f;
+          ls01 = ls23 = make_float2(0.f, 0.f);
+          const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(-mb, -mb);
 #pragma unroll
           for (int j = 0; j < C::HALF / 2; j += 2) {
-            const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * j]), scale_log2, -mb));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * j + 1]), scale_log2, -mb));
-            const float p2 = ex2_approx(fmaf(__uint_as_float(sr[2 * j + 2]), scale_log2, -mb));
-            const float p3 = ex2_approx(fmaf(__uint_as_float(sr[2 * j + 3]), scale_log2, -mb));
-            ls0 += p0;
-            ls1 += p1;
-            ls2 += p2;
-            ls3 += p3;
-            pk[j] = pack_bf16x2(p0, p1);
-            pk[j + 1] = pack_bf16x2(p2, p3);
+            const float2 x01 = __ffma2_rn(
+                make_float2(__uint_as_float(sr[2 * j]), __uint_as_float(sr[2 * j + 1])), sc2, nm2);
+            const float2 x23 = __ffma2_rn(
+                make_float2(__uint_as_float(sr[2 * j + 2]), __uint_as_float(sr[2 * j + 3])), sc2, nm2);
+            const float2 p01 = make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
+            const float2 p23 = make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
+            ls01 = __fadd2_rn(ls01, p01);
+            ls23 = __fadd2_rn(ls23, p23);
+            pk[j] = pack_bf16x2(p01.x, p01.y);
+            pk[j + 1] = pack_bf16x2(p23.x, p23.y);
           }
         };
         // Speculate that the running max stays (it does unless a row's max grows
         // by more than kRescaleTau): P first, the other half's maxima after.
         const bool spec = __all_sync(0xffffffffu, m_use != -INFINITY);
         if (spec) compute_p(m_use);
-        if (warp == 0 && lane == 0) AJVP_EVX(g, 11, ls3);
+        if (warp == 0 && lane == 0) AJVP_EVX(g, 11, ls23.y);
         // row maximum over both halves of the tile
         float their_max;
         if (!read_max(their_max)) { ok = false; break; }
@@ -830,7 +833,7 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
             tmem_st32(tT + 32 * c, a);
           }
         }
-        l += (ls0 + ls1) + (ls2 + ls3);
+        l += (ls01.x + ls01.y) + (ls23.x + ls23.y);
         if (warp == 0 && lane == 0) AJVP_EV(g, 7);
 
         if (!wwait(ts_full, ts_ph)) { ok = false; break; }
@@ -849,29 +852,31 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
         __syncwarp();
         if (lane == 0) arrive_leader(p_full);
         uint32_t uk[C::HALF / 2];
-        float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
-        // u = p s tS' for keys [32 h, 32 h + 32) of this warpgroup's half tile
+        float2 d01 = make_float2(0.f, 0.f), d23 = make_float2(0.f, 0.f);
+        const float2 sc2 = make_float2(scale, scale);
+        // u = p s tS' for keys [32 h, 32 h + 32) of this warpgroup's half
+        // tile, on pairs of floats (FMUL2, FADD2)
         auto u_half = [&](int h) {
 #pragma unroll
           for (int j = 0; j < 16; j += 2) {
             const uint32_t pa = pk[16 * h + j], pb = pk[16 * h + j + 1];
-            const float u0 = bf16lo_to_f32(pa) * scale * __uint_as_float(v[2 * j]);
-            const float u1 = bf16hi_to_f32(pa) * scale * __uint_as_float(v[2 * j + 1]);
-            const float u2 = bf16lo_to_f32(pb) * scale * __uint_as_float(v[2 * j + 2]);
-            const float u3 = bf16hi_to_f32(pb) * scale * __uint_as_float(v[2 * j + 3]);
-            d0 += u0;
-            d1 += u1;
-            d2 += u2;
-            d3 += u3;
-            uk[16 * h + j] = pack_bf16x2(u0, u1);
-            uk[16 * h + j + 1] = pack_bf16x2(u2, u3);
+            const float2 u01 = __fmul2_rn(
+                __fmul2_rn(make_float2(bf16lo_to_f32(pa), bf16hi_to_f32(pa)), sc2),
+                make_float2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1])));
+            const float2 u23 = __fmul2_rn(
+                __fmul2_rn(make_float2(bf16lo_to_f32(pb), bf16hi_to_f32(pb)), sc2),
+                make_float2(__uint_as_float(v[2 * j + 2]), __uint_as_float(v[2 * j + 3])));
+            d01 = __fadd2_rn(d01, u01);
+            d23 = __fadd2_rn(d23, u23);
+            uk[16 * h + j] = pack_bf16x2(u01.x, u01.y);
+            uk[16 * h + j + 1] = pack_bf16x2(u23.x, u23.y);
           }
         };
         u_half(0);
         tmem_ld32(tTS + 32, v);
         tmem_wait_ld();
         u_half(1);
-        dsum += (d0 + d1) + (d2 + d3);
+        dsum += (d01.x + d01.y) + (d23.x + d23.y);
         tmem_st32(tTS + 32, uk);
         tmem_wait_st();
         tc_fence_before();

@@ -50,6 +50,7 @@ constexpr float kLog2eF = 1.4426950408889634f;
 
 struct BwdTcParams {
   CUtensorMap map_q, map_k, map_v, map_do;  // [B, L, H, d] bf16, boxes of 64 columns x 128 rows
+  CUtensorMap map_q64, map_do64;            // the same for Q and dO, boxes of 64 x 64 rows
   const __nv_bfloat16* o;
   const __nv_bfloat16* dout;
   const float* lse;
@@ -115,11 +116,12 @@ struct ColScan {
   uint32_t vis, full;
 };
 
-__device__ __forceinline__ void col_scan_load(const MaskSpec& m, ColScan& cs) {
+// bq: rows of a query tile (the key tiles are kBB wide)
+__device__ __forceinline__ void col_scan_load(const MaskSpec& m, ColScan& cs, int bq) {
   const int qt = cs.base + static_cast<int>(threadIdx.x & 31);
   bool v = false, f = false;
   if (qt < cs.n_qt) {
-    const TileSched s = make_tile_sched(m, qt, kBB, kBB);
+    const TileSched s = make_tile_sched(m, qt, bq, kBB);
     v = (cs.kt >= s.t1_begin && cs.kt < s.t1_end) || (cs.kt >= s.t2_begin && cs.kt < s.t2_end);
     f = v && s.full(cs.kt);
   }
@@ -127,19 +129,21 @@ __device__ __forceinline__ void col_scan_load(const MaskSpec& m, ColScan& cs) {
   cs.full = __ballot_sync(0xffffffffu, f);
 }
 
-__device__ __forceinline__ void col_scan_start(const MaskSpec& m, ColScan& cs, int kt, int n_qt) {
+__device__ __forceinline__ void col_scan_start(const MaskSpec& m, ColScan& cs, int kt, int n_qt,
+                                               int bq) {
   cs.kt = kt;
   cs.n_qt = n_qt;
   cs.base = 0;
-  col_scan_load(m, cs);
+  col_scan_load(m, cs, bq);
 }
 
 // The next visited query tile and whether every pair in it is admissible.
-__device__ __forceinline__ bool col_next(const MaskSpec& m, ColScan& cs, int& qt, bool& full) {
+__device__ __forceinline__ bool col_next(const MaskSpec& m, ColScan& cs, int& qt, bool& full,
+                                         int bq) {
   while (cs.vis == 0) {
     cs.base += 32;
     if (cs.base >= cs.n_qt) return false;
-    col_scan_load(m, cs);
+    col_scan_load(m, cs, bq);
   }
   const int bit = __ffs(cs.vis) - 1;
   qt = cs.base + bit;
@@ -164,20 +168,43 @@ __device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const uint32_
 }
 
 // ---------------------------------------------------------------- dK, dV
+// Query tiles of 64 rows: a stage is a quarter of the 128-key block's
+// operands, so the rings hold several tiles ahead of the MMAs (the loads
+// come from L2 and take a few thousand cycles to land), and TMEM holds two
+// tiles of S^T and dP^T, so the next tile's scores run while the softmax
+// turns the current ones into P^T and dS^T.
+constexpr int kBQ = 64;  // query rows per dK/dV tile
+
 template <int D>
 struct DkdvCfg {
   static constexpr int CH = D / 64;
-  static constexpr int TILE = kBB * D * 2;            // bytes of a [128 x D] bf16 tile
-  static constexpr int NP = D == 128 ? 2 : 5;          // stages: Q, dO, LSE log2 e, D of a query tile
-  static constexpr int STAGE = 2 * TILE + 2 * kBB * 4;
-  static constexpr int DATA = 2 * TILE + NP * STAGE;   // K, V resident, then the stages
-  static constexpr int NBAR = 2 * NP + 8;
+  static constexpr int KTILE = kBB * D * 2;           // bytes of a [128 x D] tile (K, V)
+  static constexpr int QTILE = kBQ * D * 2;           // bytes of a [64 x D] tile (Q, dO)
+  static constexpr int QSLOT = QTILE + 1024;          // Q, then LSE log2 e [64] and D [64]
+  static constexpr int NQ = D == 128 ? 5 : 8;         // Q ring slots (released after dK)
+  static constexpr int ND = D == 128 ? 4 : 8;         // dO ring slots (released after dV)
+  static constexpr int DATA = 2 * KTILE + NQ * QSLOT + ND * QTILE;
+  static constexpr int NBAR = 2 * NQ + 2 * ND + 12;
   static constexpr int BYTES = 1024 + DATA + NBAR * 8 + 16;
-  // TMEM columns: S^T (P^T over its first half per warpgroup), dP^T (dS^T likewise), dV, dK
+  // TMEM columns: S^T of tiles 0, 1 (mod 2), dP^T of tiles 0, 1, dV, dK. In a
+  // warpgroup's 32 columns of a buffer, bf16 P^T (dS^T) sits over the first 16.
   static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 256 + D, TM_COLS = 512;
-  static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte alignment of swizzled tiles");
+  static_assert(QSLOT % 1024 == 0 && QTILE % 1024 == 0, "1024-byte aligned swizzled tiles");
   static_assert(BYTES <= 232448, "shared memory budget");
 };
+
+// Value MMA of the dK/dV kernel: D[tmem] (+)= A[tmem] B, A a bf16 [128 x 64]
+// tile in TMEM in which warpgroup w holds queries [32 w, 32 w + 32) packed in
+// its first 16 columns, B a [64 queries x D] tile read MN-major.
+template <bool Dummy = true>
+__device__ __forceinline__ void mma_values_q64(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem,
+                                               uint32_t idesc, bool accumulate) {
+  const uint64_t db = smem_desc_sw128(b_smem, kBQ * 128, 1024);
+#pragma unroll
+  for (int ks = 0; ks < kBQ / 16; ++ks)
+    umma_ts(d_tmem, a_tmem + 32 * (ks >> 1) + (ks & 1) * 8, db + ((ks * 16 * 128) >> 4), idesc,
+            (accumulate || ks > 0) ? 1u : 0u);
+}
 
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_tc_kernel(const __grid_constant__ BwdTcParams p) {
@@ -186,18 +213,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_tc_kernel(const __gri
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sK = smem;
-  uint8_t* sV = smem + C::TILE;
-  uint8_t* sStage = smem + 2 * C::TILE;
+  uint8_t* sV = smem + C::KTILE;
+  uint8_t* sQ = smem + 2 * C::KTILE;                 // [NQ] Q slots
+  uint8_t* sDO = sQ + C::NQ * C::QSLOT;              // [ND] dO slots
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::DATA);
-  uint64_t* full = bars;             // [NP] stage landed
-  uint64_t* empty = bars + C::NP;    // [NP] stage consumed
-  uint64_t* kv_full = bars + 2 * C::NP;
-  uint64_t* s_full = kv_full + 1;    // S^T of the current tile in TMEM
-  uint64_t* dp_full = kv_full + 2;   // dP^T of the current tile in TMEM
-  uint64_t* p_full = kv_full + 3;    // P^T (bf16) written
-  uint64_t* ds_full = kv_full + 4;   // dS^T (bf16) written
-  uint64_t* acc_full = kv_full + 5;  // dK, dV complete
-  uint64_t* drain = kv_full + 6;
+  uint64_t* q_full = bars;                           // [NQ]
+  uint64_t* q_empty = bars + C::NQ;                  // [NQ]
+  uint64_t* do_full = bars + 2 * C::NQ;              // [ND]
+  uint64_t* do_empty = do_full + C::ND;              // [ND]
+  uint64_t* kv_full = do_empty + C::ND;
+  uint64_t* s_full = kv_full + 1;    // [2] S^T of the tile in buffer b
+  uint64_t* dp_full = kv_full + 3;   // [2] dP^T
+  uint64_t* p_full = kv_full + 5;    // [2] P^T (bf16) written
+  uint64_t* ds_full = kv_full + 7;   // [2] dS^T (bf16) written
+  uint64_t* acc_full = kv_full + 9;  // dK, dV complete
+  uint64_t* drain = kv_full + 10;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -206,6 +236,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_tc_kernel(const __gri
   const int bh = blockIdx.x / p.n_kt;
   const int kt = blockIdx.x - bh * p.n_kt;
   const int b = bh / p.H, h = bh - b * p.H;
+  const int n_q64 = p.Lp / kBQ;
   MaskSpec mask = p.mask;
   mask.groups = p.groups;
   auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
@@ -213,15 +244,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_tc_kernel(const __gri
   };
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::NP; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
+    for (int i = 0; i < C::NQ; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+    }
+    for (int i = 0; i < C::ND; ++i) {
+      mbar_init(&do_full[i], 1);
+      mbar_init(&do_empty[i], 1);
     }
     mbar_init(kv_full, 1);
-    mbar_init(s_full, 1);
-    mbar_init(dp_full, 1);
-    mbar_init(p_full, 8);
-    mbar_init(ds_full, 8);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&dp_full[i], 1);
+      mbar_init(&p_full[i], 8);
+      mbar_init(&ds_full[i], 8);
+    }
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -238,14 +275,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_tc_kernel(const __gri
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
-    tma_prefetch_desc(&p.map_q);
+    // K and V of the block, then per visited query tile g: Q_g with its LSE
+    // and D rows (Q ring), dO_g (dO ring).
+    tma_prefetch_desc(&p.map_q64);
     tma_prefetch_desc(&p.map_k);
     tma_prefetch_desc(&p.map_v);
-    tma_prefetch_desc(&p.map_do);
+    tma_prefetch_desc(&p.map_do64);
     const uint64_t keep = l2_policy_evict_last();   // Q, dO: read by every key block of the head
     const uint64_t once = l2_policy_evict_first();  // K, V: this CTA only
     if (elect_one()) {
-      mbar_arrive_expect_tx(kv_full, 2 * C::TILE);
+      mbar_arrive_expect_tx(kv_full, 2 * C::KTILE);
 #pragma unroll
       for (int c = 0; c < C::CH; ++c) {
         tma_load_4d_hint(sK + c * kBB * 128, &p.map_k, kv_full, c * 64, h, kt * kBB, b, once);
@@ -257,93 +296,100 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_tc_kernel(const __gri
     const float* d_row = p.scratch + static_cast<size_t>(bh) * p.Lp;
     const float* l_row = p.scratch + total + static_cast<size_t>(bh) * p.Lp;
     ColScan cs;
-    col_scan_start(mask, cs, kt, p.n_qt);
-    uint32_t g = 0;
+    col_scan_start(mask, cs, kt, n_q64, kBQ);
+    int qn = 0, dn = 0;  // Q and dO tiles issued
     bool ok = true;
     int qt;
     bool fl;
-    while (col_next(mask, cs, qt, fl)) {
-      const uint32_t st = g % C::NP;
-      if (!wwait(&empty[st], ((g / C::NP) & 1) ^ 1)) { ok = false; break; }
-      uint8_t* stg = sStage + st * C::STAGE;
+    while (col_next(mask, cs, qt, fl, kBQ)) {
+      const int g = qn;
+      const uint32_t sq = g % C::NQ, sd = g % C::ND;
+      if (!wwait(&q_empty[sq], ((g / C::NQ) & 1) ^ 1)) { ok = false; break; }
+      uint8_t* qs = sQ + sq * C::QSLOT;
       if (elect_one()) {
-        mbar_arrive_expect_tx(&full[st], C::STAGE);
+        mbar_arrive_expect_tx(&q_full[sq], C::QTILE + 2 * kBQ * 4);
 #pragma unroll
-        for (int c = 0; c < C::CH; ++c) {
-          tma_load_4d_hint(stg + c * kBB * 128, &p.map_q, &full[st], c * 64, h, qt * kBB, b, keep);
-          tma_load_4d_hint(stg + C::TILE + c * kBB * 128, &p.map_do, &full[st], c * 64, h, qt * kBB,
-                           b, keep);
-        }
-        bulk_load(stg + 2 * C::TILE, l_row + qt * kBB, kBB * 4, &full[st]);
-        bulk_load(stg + 2 * C::TILE + kBB * 4, d_row + qt * kBB, kBB * 4, &full[st]);
+        for (int c = 0; c < C::CH; ++c)
+          tma_load_4d_hint(qs + c * kBQ * 128, &p.map_q64, &q_full[sq], c * 64, h, qt * kBQ, b, keep);
+        bulk_load(qs + C::QTILE, l_row + qt * kBQ, kBQ * 4, &q_full[sq]);
+        bulk_load(qs + C::QTILE + kBQ * 4, d_row + qt * kBQ, kBQ * 4, &q_full[sq]);
       }
       __syncwarp();
-      ++g;
+      qn = g + 1;
+      if (!wwait(&do_empty[sd], ((g / C::ND) & 1) ^ 1)) { ok = false; break; }
+      if (elect_one()) {
+        mbar_arrive_expect_tx(&do_full[sd], C::QTILE);
+#pragma unroll
+        for (int c = 0; c < C::CH; ++c)
+          tma_load_4d_hint(sDO + sd * C::QTILE + c * kBQ * 128, &p.map_do64, &do_full[sd], c * 64, h,
+                           qt * kBQ, b, keep);
+      }
+      __syncwarp();
+      dn = g + 1;
     }
     if (!ok && lane == 0) {
       // Abort: let every copy already issued land before the CTA exits.
       mbar_wait_drain(kv_full, 0, 200000000ull);
-      for (uint32_t s = 0; s < C::NP && s < g; ++s) {
-        const uint32_t last = g - 1 - ((g - 1 + C::NP - s) % C::NP);
-        mbar_wait_drain(&full[s], (last / C::NP) & 1, 200000000ull);
-      }
+      for (int j = qn - 1; j >= 0 && j >= qn - C::NQ; --j)
+        mbar_wait_drain(&q_full[j % C::NQ], (j / C::NQ) & 1, 200000000ull);
+      for (int j = dn - 1; j >= 0 && j >= dn - C::ND; --j)
+        mbar_wait_drain(&do_full[j % C::ND], (j / C::ND) & 1, 200000000ull);
     }
     __syncwarp();
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    // Per query tile g (stage g % NP): dV_g, S^T_{g+1}, dK_g, dP^T_{g+1}.
-    // P^T_g sits over S^T_g's columns and dS^T_g over dP^T_g's; one thread's
-    // tcgen05.mma execute in issue order, so S^T_{g+1} follows dV_g's reads
-    // of P^T_g and dP^T_{g+1} follows dK_g's reads of dS^T_g.
-    const uint32_t idesc_s = idesc_bf16_f32(128, kBB, 0);
+    // Scores of tile g go to TMEM buffer g % 2. Per tile g: dV_g (after
+    // P^T_g), dK_g (after dS^T_g), then S^T_{g+2} and dP^T_{g+2} into the same
+    // buffer: one thread's tcgen05.mma execute in issue order, so they follow
+    // dV_g's and dK_g's reads of P^T_g and dS^T_g. Meanwhile the softmax
+    // works on tile g+1, whose scores were issued a tile earlier.
+    const uint32_t idesc_s = idesc_bf16_f32(128, kBQ, 0);
     const uint32_t idesc_v = idesc_bf16_f32(128, D, 1);
-    const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aSt = smem_u32(sStage);
-    auto st_q = [&](uint32_t g) { return aSt + (g % C::NP) * C::STAGE; };
-    auto st_do = [&](uint32_t g) { return st_q(g) + C::TILE; };
-    auto st_full = [&](uint32_t g) { return &full[g % C::NP]; };
-    auto st_ph = [&](uint32_t g) { return (g / C::NP) & 1; };
-    auto test = [&](uint64_t* bar, uint32_t parity) -> bool {
-      return __shfl_sync(0xffffffffu, mbar_test_wait(bar, parity) ? 1 : 0, 0) != 0;
+    const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
+    const uint32_t aQ0 = smem_u32(sQ), aD0 = smem_u32(sDO);
+    auto q_addr = [&](int g) { return aQ0 + (g % C::NQ) * C::QSLOT; };
+    auto do_addr = [&](int g) { return aD0 + (g % C::ND) * C::QTILE; };
+    // scores of tile j into buffer j % 2
+    auto issue_scores = [&](int j) -> bool {
+      const int bf = j & 1;
+      if (!wwait(&q_full[j % C::NQ], (j / C::NQ) & 1)) return false;
+      tc_fence_after();
+      mma_scores<D, kBB, kBQ, false>(tmem + C::TM_S + 64 * bf, aK, q_addr(j), idesc_s, false);
+      umma_commit(&s_full[bf]);
+      if (!wwait(&do_full[j % C::ND], (j / C::ND) & 1)) return false;
+      tc_fence_after();
+      mma_scores<D, kBB, kBQ, false>(tmem + C::TM_DP + 64 * bf, aV, do_addr(j), idesc_s, false);
+      umma_commit(&dp_full[bf]);
+      return true;
     };
     ColScan cs;
-    col_scan_start(mask, cs, kt, p.n_qt);
+    col_scan_start(mask, cs, kt, n_q64, kBQ);
     int qt;
     bool fl;
-    if (col_next(mask, cs, qt, fl)) {
-      bool ok = wwait(kv_full, 0) && wwait(st_full(0), 0);
-      if (ok) {
-        tc_fence_after();
-        mma_scores<D, kBB, kBB, false>(tmem + C::TM_S, aK, st_q(0), idesc_s, false);
-        umma_commit(s_full);
-        mma_scores<D, kBB, kBB, false>(tmem + C::TM_DP, aV, st_do(0), idesc_s, false);
-        umma_commit(dp_full);
-      }
-      for (uint32_t g = 0; ok; ++g) {
-        const bool has_next = col_next(mask, cs, qt, fl);
-        const uint32_t ph = g & 1;
-        bool rdy_n = false, rdy_ds = false;
-        if (!wwait(p_full, ph)) break;
-        tc_fence_after();
-        mma_values_split<kBB, false, 3>(tmem + C::TM_DV, tmem + C::TM_S, st_do(g), idesc_v, g > 0, [&] {
-          if (has_next) rdy_n = test(st_full(g + 1), st_ph(g + 1));
-        });
-        if (has_next) {
-          if (!rdy_n && !wwait(st_full(g + 1), st_ph(g + 1))) break;
-          tc_fence_after();
-          mma_scores<D, kBB, kBB, false, D / 32>(tmem + C::TM_S, aK, st_q(g + 1), idesc_s, false,
-                                                [&] { rdy_ds = test(ds_full, ph); });
-          umma_commit(s_full);
-        }
-        if (!rdy_ds && !wwait(ds_full, ph)) break;
-        tc_fence_after();
-        mma_values_split<kBB, false>(tmem + C::TM_DK, tmem + C::TM_DP, st_q(g), idesc_v, g > 0);
-        umma_commit(&empty[g % C::NP]);
-        if (!has_next) {
-          umma_commit(acc_full);
-          break;
-        }
-        mma_scores<D, kBB, kBB, false>(tmem + C::TM_DP, aV, st_do(g + 1), idesc_s, false);
-        umma_commit(dp_full);
+    int n_tiles = 0;  // tiles found so far by the scan (the MMA warp runs two ahead)
+    bool ok = true;
+    if (wwait(kv_full, 0)) {
+      for (; n_tiles < 2 && col_next(mask, cs, qt, fl, kBQ); ++n_tiles)
+        if (!issue_scores(n_tiles)) { ok = false; break; }
+    } else {
+      ok = false;
+    }
+    for (int g = 0; ok && g < n_tiles; ++g) {
+      const int bf = g & 1;
+      const uint32_t ph = (g >> 1) & 1;
+      if (!wwait(&p_full[bf], ph)) break;
+      tc_fence_after();
+      mma_values_q64(tmem + C::TM_DV, tmem + C::TM_S + 64 * bf, do_addr(g), idesc_v, g > 0);
+      umma_commit(&do_empty[g % C::ND]);
+      if (!wwait(&ds_full[bf], ph)) break;
+      tc_fence_after();
+      mma_values_q64(tmem + C::TM_DK, tmem + C::TM_DP + 64 * bf, q_addr(g), idesc_v, g > 0);
+      umma_commit(&q_empty[g % C::NQ]);
+      if (col_next(mask, cs, qt, fl, kBQ)) {
+        if (!issue_scores(n_tiles)) break;
+        ++n_tiles;
+      } else if (g == n_tiles - 1) {
+        umma_commit(acc_full);
       }
     }
     // Every MMA issued so far completes before TMEM is released.
@@ -353,65 +399,57 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_tc_kernel(const __gri
   } else {
     // ------------------------------------------------------------ softmax + epilogue
     // Thread (wg, sub, lane) owns key row 32 sub + lane (its TMEM lane) and the
-    // query columns [64 wg, 64 wg + 64) of every tile.
+    // query columns [32 wg, 32 wg + 32) of every 64-row query tile.
     const int wg = warp >> 2, sub = warp & 3;
     const int row = sub * 32 + lane;
     const int key = kt * kBB + row;
     const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
-    const uint32_t tS = tmem + lane_off + C::TM_S + 64 * wg;
-    const uint32_t tDP = tmem + lane_off + C::TM_DP + 64 * wg;
     const uint32_t tDV = tmem + lane_off + C::TM_DV + (D / 2) * wg;
     const uint32_t tDK = tmem + lane_off + C::TM_DK + (D / 2) * wg;
-    const float sl2 = p.scale_log2;
+    const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
     ColScan cs;
-    col_scan_start(mask, cs, kt, p.n_qt);
-    uint32_t g = 0;
+    col_scan_start(mask, cs, kt, n_q64, kBQ);
+    int g = 0;
     bool ok = true;
     int qt;
     bool fl;
-    while (col_next(mask, cs, qt, fl)) {
-      const uint32_t st = g % C::NP, ph = g & 1;
-      const float* lse2 = reinterpret_cast<const float*>(sStage + st * C::STAGE + 2 * C::TILE) + 64 * wg;
-      const float* dd = lse2 + kBB;
-      // the stage's LSE and D are read from shared memory: observe its copies
-      if (!wwait(&full[st], (g / C::NP) & 1)) { ok = false; break; }
-      if (!wwait(s_full, ph)) { ok = false; break; }
+    while (col_next(mask, cs, qt, fl, kBQ)) {
+      const int bf = g & 1;
+      const uint32_t ph = (g >> 1) & 1;
+      const uint32_t tS = tmem + lane_off + C::TM_S + 64 * bf + 32 * wg;
+      const uint32_t tDP = tmem + lane_off + C::TM_DP + 64 * bf + 32 * wg;
+      const float* lse2 =
+          reinterpret_cast<const float*>(sQ + (g % C::NQ) * C::QSLOT + C::QTILE) + 32 * wg;
+      const float* dd = lse2 + kBQ;
+      // the tile's LSE and D are read from shared memory: observe its copies
+      if (!wwait(&q_full[g % C::NQ], (g / C::NQ) & 1)) { ok = false; break; }
+      if (!wwait(&s_full[bf], ph)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sr[64];
-      tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      uint32_t sr[32];
+      tmem_ld32(tS, sr);
       tmem_wait_ld();
       if (!fl) {
-        // Admissible query columns of this key: row by row, since the mask is
-        // given per query row; ranges are recomputed only where a new row group starts.
-        uint32_t m0 = 0, m1 = 0;
-        int i = qt * kBB + 64 * wg;
+        // Admissible query columns of this key, row group by row group.
+        uint32_t m = 0;
+        int i = qt * kBQ + 32 * wg;
         RowRange rr = row_range(mask, i);
         int nxt = next_group_start(mask, i);
 #pragma unroll 1
-        for (int c = 0; c < 64; ++c, ++i) {
+        for (int c = 0; c < 32; ++c, ++i) {
           if (i >= nxt) {
             rr = row_range(mask, i);
             nxt = next_group_start(mask, i);
           }
-          const uint32_t a = row_allows(rr, key) ? 1u : 0u;
-          if (c < 32)
-            m0 |= a << c;
-          else
-            m1 |= a << (c - 32);
+          m |= (row_allows(rr, key) ? 1u : 0u) << c;
         }
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          if (!((m0 >> j) & 1u)) sr[j] = __float_as_uint(-INFINITY);
-          if (!((m1 >> j) & 1u)) sr[32 + j] = __float_as_uint(-INFINITY);
-        }
+        for (int j = 0; j < 32; ++j)
+          if (!((m >> j) & 1u)) sr[j] = __float_as_uint(-INFINITY);
       }
       // P^T = 2^(S^T s log2 e - LSE_i log2 e): 0 where masked or past L
-      // scalings on pairs of floats (FFMA2); S^T s log2 e - LSE_i log2 e
-      uint32_t pk[32];
-      const float2 sc2 = make_float2(sl2, sl2);
+      uint32_t pk[16];
 #pragma unroll
-      for (int j = 0; j < 64; j += 4) {
+      for (int j = 0; j < 32; j += 4) {
         const float4 l4 = *reinterpret_cast<const float4*>(lse2 + j);
         const float2 x01 = __ffma2_rn(make_float2(__uint_as_float(sr[j]), __uint_as_float(sr[j + 1])),
                                       sc2, make_float2(-l4.x, -l4.y));
@@ -426,37 +464,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_tc_kernel(const __gri
         pk[j / 2] = pack_bf16x2(p0, p1);
         pk[j / 2 + 1] = pack_bf16x2(p2, p3);
       }
-      tmem_st32(tS, pk);
+      tmem_st16(tS, pk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
-      // dS^T = P^T (dP^T - D_i), over the first half of this warpgroup's dP^T slice
-      if (!wwait(dp_full, ph)) { ok = false; break; }
+      if (lane == 0) mbar_arrive(&p_full[bf]);
+      // dS^T = P^T (dP^T - D_i) on pairs of floats, over the first half of
+      // this warpgroup's dP^T columns
+      if (!wwait(&dp_full[bf], ph)) { ok = false; break; }
       tc_fence_after();
       uint32_t v[32];
       tmem_ld32(tDP, v);
       tmem_wait_ld();
-      // dS^T = P^T (dP^T - D_i) on pairs of floats (FADD2, FMUL2)
-      auto ds_pair = [&](int c, uint32_t v0, uint32_t v1, float2 d2) -> uint32_t {
-        const float2 ds = __fmul2_rn(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])),
-                                     __fadd2_rn(make_float2(__uint_as_float(v0), __uint_as_float(v1)),
+#pragma unroll
+      for (int j = 0; j < 32; j += 2) {
+        const float2 d2 = *reinterpret_cast<const float2*>(dd + j);
+        const float2 ds = __fmul2_rn(make_float2(__uint_as_float(sr[j]), __uint_as_float(sr[j + 1])),
+                                     __fadd2_rn(make_float2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])),
                                                 make_float2(-d2.x, -d2.y)));
-        return pack_bf16x2(ds.x, ds.y);
-      };
-#pragma unroll
-      for (int j = 0; j < 32; j += 2)
-        pk[j / 2] = ds_pair(j, v[j], v[j + 1], *reinterpret_cast<const float2*>(dd + j));
-      tmem_ld32(tDP + 32, v);
-      tmem_wait_ld();
-#pragma unroll
-      for (int j = 0; j < 32; j += 2)
-        pk[16 + j / 2] = ds_pair(32 + j, v[j], v[j + 1], *reinterpret_cast<const float2*>(dd + 32 + j));
-      tmem_st32(tDP, pk);
+        pk[j / 2] = pack_bf16x2(ds.x, ds.y);
+      }
+      tmem_st16(tDP, pk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(ds_full);
+      if (lane == 0) mbar_arrive(&ds_full[bf]);
       ++g;
     }
     // ---------------- epilogue: dV, s dK of this key (zero if no query sees it)
@@ -884,7 +916,9 @@ int bwd_tc_launch(const BwdTcArgs& a, cudaStream_t stream) {
   if (!encode_bf16_rows_map(&p.map_q, a.q, a.B, a.L, a.H, a.d, kBB) ||
       !encode_bf16_rows_map(&p.map_k, a.k, a.B, a.L, a.H, a.d, kBB) ||
       !encode_bf16_rows_map(&p.map_v, a.v, a.B, a.L, a.H, a.d, kBB) ||
-      !encode_bf16_rows_map(&p.map_do, a.dout, a.B, a.L, a.H, a.d, kBB))
+      !encode_bf16_rows_map(&p.map_do, a.dout, a.B, a.L, a.H, a.d, kBB) ||
+      !encode_bf16_rows_map(&p.map_q64, a.q, a.B, a.L, a.H, a.d, kBQ) ||
+      !encode_bf16_rows_map(&p.map_do64, a.dout, a.B, a.L, a.H, a.d, kBQ))
     return ATTN_JVP_ERR_CUDA;
   p.o = static_cast<const __nv_bfloat16*>(a.o);
   p.dout = static_cast<const __nv_bfloat16*>(a.dout);

@@ -18,19 +18,22 @@
 //      serves as scratch until launch 3 overwrites it. Padded rows i >= L get
 //      D = 0 and LSE = +inf, so their P is exactly 0.
 //   2. bwd_dkdv_tc_kernel: one CTA per 128 keys of a (batch, head). dK and dV
-//      stay in TMEM while the CTA streams the query tiles whose key-tile
-//      schedule lists this key tile (the forward's schedule, transposed):
-//        S^T = K Q^T, dP^T = V dO^T            (SS MMAs, K and V resident)
+//      stay in TMEM while the CTA streams, 64 query rows at a time, the query
+//      tiles whose key-tile schedule lists this key tile (the forward's
+//      schedule, transposed), from separate Q and dO rings:
+//        S^T = K Q^T, dP^T = V dO^T            (SS MMAs, K and V resident,
+//                                               two TMEM buffers of each)
 //        P^T, dS^T in registers (bf16 copies back to TMEM over S^T, dP^T)
 //        dV += P^T dO, dK += dS^T Q            (A operand read from TMEM)
 //   3. bwd_dq_tc_kernel: one CTA per 128 query rows, over the key tiles of the
-//      forward's schedule:
+//      forward's schedule, from separate K and V rings:
 //        S = Q K^T, dP = dO V^T (two dP buffers), dS in registers,
 //        dQ += dS K                            (A operand read from TMEM)
 //      It forms D_i itself from O and dO, since it overwrites the scratch.
-// Warp roles (320 threads): warps 0-7 two "softmax" warpgroups (each owns 64
-// of a tile's 128 columns), warp 8 TMA producer, warp 9 MMA issuer and TMEM
-// allocator. Every wait is bounded (see ptx.cuh).
+// Warp roles (320 threads): warps 0-7 two "softmax" warpgroups (each owns half
+// of a tile's columns: 32 of 64 in the dK/dV kernel, 64 of 128 in the dQ
+// kernel), warp 8 TMA producer, warp 9 MMA issuer and TMEM allocator. Every
+// wait is bounded (see ptx.cuh).
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -468,7 +471,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_tc_kernel(const __gri
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[bf]);
+      mbar_arrive_if(&p_full[bf], lane == 0);
       // dS^T = P^T (dP^T - D_i) on pairs of floats, over the first half of
       // this warpgroup's dP^T columns
       if (!wwait(&dp_full[bf], ph)) { ok = false; break; }
@@ -488,7 +491,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_tc_kernel(const __gri
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ds_full[bf]);
+      mbar_arrive_if(&ds_full[bf], lane == 0);
       ++g;
     }
     // ---------------- epilogue: dV, s dK of this key (zero if no query sees it)
@@ -784,7 +787,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_tc_kernel(const __grid_
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(s_free);  // S_j is in registers: S_{j+1} may be written
+      mbar_arrive_if(s_free, lane == 0);  // S_j is in registers: S_{j+1} may be written
       if (!full_tile) {
         const int k0 = kt * kBB + 64 * wg;
         const int s1 = min(max(rr.a0 - k0, 0), 64), e1 = min(max(rr.a1 - k0, 0), 64);
@@ -830,7 +833,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_tc_kernel(const __grid_
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ds_full[idx & 1]);
+      mbar_arrive_if(&ds_full[idx & 1], lane == 0);
     }
     // ---------------- epilogue: s dQ of this row
     if (ok) {

@@ -269,6 +269,13 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
     else
       mbar_arrive(bar);
   };
+  // One arrival per warp (lane 0), branch-free.
+  auto arrive_leader_warp = [&](uint64_t* bar) {
+    if (PAIR && rank != 0)
+      mbar_arrive_remote_if(leader_addr(bar), lane == 0);
+    else
+      mbar_arrive_if(bar, lane == 0);
+  };
   auto bwait = [&](uint64_t* bar, uint32_t parity) -> bool {
     return mbar_wait(bar, parity, abort_flag, p.status, p.wait_ns);
   };
@@ -655,39 +662,31 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
     // arrived on s_free, which each does after reading this value. Bounded spin.
     // The swap is split: publish this warpgroup's maxima, compute P with the
     // running max meanwhile, then read the other's (normally long there).
+    // Every lane takes part (same words, one request per access), so that
+    // the warp does not diverge.
     auto publish_max = [&](float mine) {
       *my_x = mine;
-      __syncwarp();
+      __syncwarp();  // every lane's value before any lane's flag
       ++xseq;
-      if (lane == 0) {
-        __threadfence_block();
-        *my_flag = xseq;
-      }
-      __syncwarp();
+      __threadfence_block();
+      *my_flag = xseq;
     };
     auto read_max = [&](float& theirs) -> bool {
-      int ok = 1;
-      if (lane == 0) {
-        uint32_t polls = 0;
-        uint64_t t0 = 0;
-        while (static_cast<int>(*other_flag - xseq) < 0) {
-          if ((++polls & 63u) == 0) {
-            if (*abort_flag) { ok = 0; break; }
-            const uint64_t now = globaltimer_ns();
-            if (t0 == 0) t0 = now;
-            if (now - t0 > p.wait_ns) {
-              *abort_flag = 1;
-              atomicOr(p.status, kStatusTimeout);
-              ok = 0;
-              break;
-            }
+      uint32_t polls = 0;
+      uint64_t t0 = 0;
+      while (__any_sync(0xffffffffu, static_cast<int>(*other_flag - xseq) < 0)) {
+        if ((++polls & 63u) == 0) {
+          if (__any_sync(0xffffffffu, *abort_flag != 0)) return false;
+          const uint64_t now = globaltimer_ns();
+          if (t0 == 0) t0 = now;
+          if (__any_sync(0xffffffffu, now - t0 > p.wait_ns)) {
+            *abort_flag = 1;
+            if (lane == 0) atomicOr(p.status, kStatusTimeout);
+            return false;
           }
         }
-        __threadfence_block();
       }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      __syncwarp();
-      if (!ok) return false;
+      __threadfence_block();
       theirs = *other_x;
       return true;
     };
@@ -790,7 +789,7 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
         // S_g is in registers and both warpgroups have read this tile's maxima:
         // the MMA warp may write S_{g+1} over S_g.
         __syncwarp();
-        if (lane == 0) arrive_leader(s_free);
+        arrive_leader_warp(s_free);
         tc_fence_after();
         const float row_max = fmaxf(my_max, their_max);
         if (warp == 0 && lane == 0) AJVP_EV(g, 6);
@@ -850,7 +849,7 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) arrive_leader(p_full);
+        arrive_leader_warp(p_full);
         uint32_t uk[C::HALF / 2];
         float2 d01 = make_float2(0.f, 0.f), d23 = make_float2(0.f, 0.f);
         const float2 sc2 = make_float2(scale, scale);
@@ -881,7 +880,7 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) arrive_leader(u_full);
+        arrive_leader_warp(u_full);
         if (warp == 0 && lane == 0) AJVP_EV(g, 9);
       }
       if (!ok) break;

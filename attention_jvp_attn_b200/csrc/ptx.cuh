@@ -113,18 +113,36 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
-// Whole-warp wait: lane 0 polls (one shared-memory request per poll instead
-// of 32), the result is broadcast, and the warp is reconverged (with memory
-// ordering to the other lanes) before any warp-collective tcgen05 instruction.
+// Whole-warp wait: every lane polls (the same barrier word: one shared-memory
+// request per poll) and the lanes decide together through warp votes, so the
+// warp never diverges and stays converged for the warp-collective tcgen05
+// instructions that follow. Bounded like mbar_wait.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           unsigned int* status,
                                           uint64_t limit_ns = kWaitTimeoutNs) {
-  int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag, status, limit_ns) ? 1 : 0;
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  __syncwarp();
-  if (!ok) *abort_flag = 1;
-  return ok != 0;
+  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 8; ++i)
+      if (__all_sync(0xffffffffu, mbar_try_wait_sleep(bar, parity, 200000u))) return true;
+    if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+    if (__any_sync(0xffffffffu, globaltimer_ns() - t0 > limit_ns)) {
+      if (status && (threadIdx.x & 31) == 0) atomicOr(status, kStatusTimeout);
+      break;
+    }
+  }
+  *abort_flag = 1;
+  return false;
+}
+
+// Arrive on `bar` from the lanes where `pred` holds, without a branch.
+__device__ __forceinline__ void mbar_arrive_if(uint64_t* bar, bool pred) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "@p mbarrier.arrive.shared::cta.b64 _, [%0];\n\t}\n" ::"r"(smem_u32(bar)),
+      "r"(static_cast<uint32_t>(pred))
+      : "memory");
 }
 
 // Wait used only while draining after an abort: bounded, never raises.
@@ -394,6 +412,15 @@ __device__ __forceinline__ bool mbar_wait_acquire_cluster(uint64_t* bar, uint32_
 // only add a wait for this thread's other memory traffic.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// The same from the lanes where `pred` holds, without a branch.
+__device__ __forceinline__ void mbar_arrive_remote_if(uint32_t cluster_addr, bool pred) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "@p mbarrier.arrive.shared::cluster.b64 _, [%0];\n\t}\n" ::"r"(cluster_addr),
+      "r"(static_cast<uint32_t>(pred))
+      : "memory");
 }
 
 // Tiled 4-D load into this CTA's shared memory whose completion (bytes) is

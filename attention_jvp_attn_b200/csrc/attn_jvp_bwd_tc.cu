@@ -234,7 +234,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_tc_kernel(const __gri
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-  const int warp = threadIdx.x >> 5;
+  const int warp = warp_uniform(static_cast<int>(threadIdx.x >> 5));
   const int lane = threadIdx.x & 31;
   const int bh = blockIdx.x / p.n_kt;
   const int kt = blockIdx.x - bh * p.n_kt;
@@ -274,7 +274,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_tc_kernel(const __gri
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem = static_cast<uint32_t>(warp_uniform(static_cast<int>(*tmem_slot)));
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
@@ -583,7 +583,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_tc_kernel(const __grid_
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-  const int warp = threadIdx.x >> 5;
+  const int warp = warp_uniform(static_cast<int>(threadIdx.x >> 5));
   const int lane = threadIdx.x & 31;
   // Items in reverse query-tile order within a head: under causal masks the
   // last query tiles see the most keys, so the longest items start first.
@@ -592,7 +592,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_tc_kernel(const __grid_
   const int b = bh / p.H, h = bh - b * p.H;
   MaskSpec mask = p.mask;
   mask.groups = p.groups;
-  const TileSched sch = make_tile_sched(mask, qt, kBB, kBB);
+  const TileSched sch = warp_uniform(make_tile_sched(mask, qt, kBB, kBB));
   const int cnt = sch.count();
   auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
     return warp_wait(bar, parity, abort_flag, p.status);
@@ -623,7 +623,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_tc_kernel(const __grid_
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem = static_cast<uint32_t>(warp_uniform(static_cast<int>(*tmem_slot)));
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer

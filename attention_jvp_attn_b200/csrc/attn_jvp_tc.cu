@@ -133,7 +133,7 @@ __device__ __forceinline__ int item_position(int k, int cta, int G) {
 
 // The unit's k-th work item (work lists), or its first item at snake round
 // >= k (k is advanced to it).
-__device__ __forceinline__ bool next_item(const TcParams& p, int cta, int G, int& k, int& pos) {
+__device__ __forceinline__ bool next_item_lane(const TcParams& p, int cta, int G, int& k, int& pos) {
   if (p.list_mode) {
     const int i = p.unit_start[cta] + k;
     if (i >= p.unit_start[cta + 1]) return false;
@@ -145,6 +145,14 @@ __device__ __forceinline__ bool next_item(const TcParams& p, int cta, int G, int
     if (pos < p.n_items) return true;
   }
   return false;
+}
+
+// next_item for a whole (converged) warp, with warp-uniform results.
+__device__ __forceinline__ bool next_item(const TcParams& p, int cta, int G, int& k, int& pos) {
+  const bool has = next_item_lane(p, cta, G, k, pos);
+  k = warp_uniform(k);
+  pos = warp_uniform(pos);
+  return warp_uniform(has ? 1 : 0) != 0;
 }
 
 __device__ __forceinline__ WorkItem decode_item(const TcParams& p, int pos) {
@@ -245,7 +253,7 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint32_t* peer_cnt = tmem_slot + 2;  // pair, leader: the peer's ring and Q copy counts
 
-  const int warp = threadIdx.x >> 5;
+  const int warp = warp_uniform(static_cast<int>(threadIdx.x >> 5));
   const int lane = threadIdx.x & 31;
 #ifdef AJVP_TRACE
   const long long trace_c0 = clock64();
@@ -336,7 +344,7 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
   else
     __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem = static_cast<uint32_t>(warp_uniform(static_cast<int>(*tmem_slot)));
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
@@ -403,7 +411,7 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
           }
         }
         ++q_issued;
-        const TileSched sch = make_tile_sched(mask, w.qt, C::BMU, C::BN);
+        const TileSched sch = warp_uniform(make_tile_sched(mask, w.qt, C::BMU, C::BN));
         const int cnt = sch.count();
         for (int idx = 0; ok && idx < cnt; ++idx) {
           const int kt = sch.tile(idx);
@@ -477,13 +485,17 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
     //   B: A (+)= P_g V_g
     //   D: T += U_g V_g                 after U_g (u_full)
     //   E: tS'_{g+1} = tQ K_{g+1}^T + Q tK_{g+1}^T
-    // C goes first when its inputs are ready (it fills the pipe while the
-    // softmax turns tS'_g into P_g), else after B, else after D. tcgen05.mma
-    // from one thread execute in order, so E (over the columns of P_g and
-    // U_g) follows every read of them. The tensor-core queue is shallow and
-    // the issuing thread waits for room, so each barrier a group depends on
-    // is tested in the middle of the group before it (the `rdy_*` flags):
-    // the test's latency then overlaps MMAs still in flight.
+    // Within an item C goes first, waiting for s_free if need be: the softmax
+    // releases S_g before P_g is ready, so the wait never delays A and B, and
+    // S_{g+1} then runs while the softmax finishes P_g and U_g. (Issuing A and
+    // B first whenever s_free was not yet there left the softmax waiting for
+    // S_{g+1} behind them.) The first tile of a new item needs the new Q, so
+    // its C comes after D. tcgen05.mma from one thread execute in order, so E
+    // (over the columns of P_g and U_g) follows every read of them. The
+    // tensor-core queue is shallow and the issuing thread waits for room, so
+    // each barrier a group depends on is tested in the middle of the group
+    // before it (the `rdy_*` flags): the test's latency then overlaps MMAs
+    // still in flight.
     // The whole warp runs this loop with identical values in every lane (one
     // elected lane issues each MMA and commit). In a pair only the leader's
     // warp 9 issues; its commits arrive on the barriers of both CTAs.
@@ -510,7 +522,7 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
       if (next_item(p, cta, G, k, pos)) {
         ++k;
         WorkItem w = decode_item(p, pos);
-        TileSched sch = make_tile_sched(mask, w.qt, C::BMU, C::BN);
+        TileSched sch = warp_uniform(make_tile_sched(mask, w.qt, C::BMU, C::BN));
         int cnt = sch.count(), idx = 0;
         uint32_t g = 0;
         // prologue: scores of the first tile (ring element 0 = KK_0)
@@ -540,7 +552,7 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
             if (has_next) {
               ++k;
               w2 = decode_item(p, pos);
-              sch2 = make_tile_sched(mask, w2.qt, C::BMU, C::BN);
+              sch2 = warp_uniform(make_tile_sched(mask, w2.qt, C::BMU, C::BN));
               cnt2 = sch2.count();
               idx2 = 0;
               new_item = true;
@@ -564,9 +576,9 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
             s_done = true;
             rdy_k = true;
           };
-          // C, early
-          if (!s_done && !new_item &&
-              (rdy_s || (test(s_free, sf_ph) && test(el_full(jk), el_ph(jk))))) {
+          // C, first within an item
+          if (!s_done && !new_item) {
+            if (!rdy_s && (!wwait(s_free, sf_ph) || !wwait(el_full(jk), el_ph(jk)))) break;
             issue_s([&] {
               rdy_v = test(el_full(jv), el_ph(jv));
               rdy_p = test(p_full, p_ph);
@@ -580,14 +592,10 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
           AJVP_EV(g, 1);
           tc_fence_after();
           mma_values_split<C::BN, PAIR>(tmem + C::TM_T, tmem + C::TM_P, aTV, idesc_v, idx > 0);
-          bool rdy_c = false;
           mma_values_split<C::BN, PAIR, 3>(tmem + C::TM_A, tmem + C::TM_P, aV, idesc_v, idx > 0, [&] {
             rdy_u = test(u_full, u_ph);
-            if (!s_done && !new_item) rdy_c = test(s_free, sf_ph) && test(el_full(jk), el_ph(jk));
           });
           AJVP_EV(g, 2);
-          // C, after B
-          if (rdy_c) issue_s([&] { if (!rdy_u) rdy_u = test(u_full, u_ph); });
           // D
           if (!rdy_u && !wwait(u_full, u_ph)) break;
           u_ph ^= 1;
@@ -599,8 +607,7 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
           commit_all(el_empty(jv));
           if (idx == cnt - 1) commit_all(acc_full);
           if (!has_next) break;
-          // C, last resort (and always for a new item's first tile, which
-          // needs the new Q)
+          // C for a new item's first tile, which needs the new Q
           if (!s_done) {
             if (new_item) {
               if (!wwait(q_full, q_ph)) break;
@@ -713,7 +720,7 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
       const WorkItem w = decode_item(p, pos);
       const int t = w.qt * C::BMU + static_cast<int>(rank) * C::BM + row;  // this thread's query row
       const RowRange rr = row_range(mask, t);
-      const TileSched sch = make_tile_sched(mask, w.qt, C::BMU, C::BN);
+      const TileSched sch = warp_uniform(make_tile_sched(mask, w.qt, C::BMU, C::BN));
       const int cnt = sch.count();
       float m_use = -INFINITY, l = 0.f, dsum = 0.f;
       for (int idx = 0; idx < cnt; ++idx, ++g) {

@@ -559,7 +559,8 @@ int attn_jvp_fwd_rope(const attn_jvp_shape* shape, const void* q, const void* k,
     if (!ptr) return ATTN_JVP_ERR_INVALID_ARGUMENT;
   for (const void* ptr : ptrs)
     if (!aligned16(ptr)) return ATTN_JVP_ERR_MISALIGNED;
-  if (shape->B * shape->L * shape->H >= (int64_t(1) << 32)) return ATTN_JVP_ERR_UNSUPPORTED;
+  // the fused rotation counts 16-byte vectors of the four tensors in 32 bits
+  if (shape->B * shape->L * shape->H * (shape->d / 2) >= (int64_t(1) << 32)) return ATTN_JVP_ERR_UNSUPPORTED;
   if (shape->dtype == ATTN_JVP_F32) {
     // fp32: the stand-alone rotation pass, then the CUDA-core attention kernel
     const int r = attn_jvp_rope(shape, q, k, tq, tk, cos, sin, q_rot, k_rot, tq_rot, tk_rot, stream);

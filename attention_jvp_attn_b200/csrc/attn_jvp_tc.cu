@@ -165,32 +165,58 @@ __device__ __forceinline__ WorkItem decode_item(const TcParams& p, int pos) {
   return w;
 }
 
-// Rotation phase of the fused rotary embedding: one warp per (token, head)
-// row at a time, each lane 16 bytes (4 pairs) of one of q, k, tq, tk.
+// Rotation phase of the fused rotary embedding: the 16-byte vectors of q, k,
+// tq and tk (in that order) are spread over every thread of the grid, and
+// each thread has kRopeInFlight of them in flight (all loads issued before the
+// first rotation), so that the phase runs at the memory's rate rather than
+// its latency. The host bounds B L H d/2 below 2^32 (the vector count).
+constexpr int kRopeInFlight = 8;
 template <int D>
 __device__ __forceinline__ void rope_phase(const TcParams& p) {
   constexpr int VPR = D / 8;  // 16-byte vectors per row of one tensor
-  const unsigned rows = static_cast<unsigned>(p.B) * p.L * p.H;
-  const unsigned warps = gridDim.x * (blockDim.x >> 5);
-  const int lane = threadIdx.x & 31;
-  for (unsigned r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
-    const unsigned t = (r / p.H) % p.L;  // token
+  const unsigned per_tensor = static_cast<unsigned>(p.B) * p.L * p.H * VPR;
+  const unsigned total = 4u * per_tensor;
+  const unsigned stride = gridDim.x * blockDim.x;
+  for (unsigned v0 = blockIdx.x * blockDim.x + threadIdx.x; v0 < total; v0 += kRopeInFlight * stride) {
+    uint4 u[kRopeInFlight];
+    float4 c[kRopeInFlight], sn[kRopeInFlight];
+    unsigned which[kRopeInFlight], e[kRopeInFlight];
 #pragma unroll
-    for (int j = lane; j < 4 * VPR; j += 32) {
-      const int which = j / VPR, col = (j % VPR) * 8;
-      const size_t off = static_cast<size_t>(r) * D + col;
-      const float4 c = *reinterpret_cast<const float4*>(p.rope_cos + static_cast<size_t>(t) * (D / 2) + col / 2);
-      const float4 sn = *reinterpret_cast<const float4*>(p.rope_sin + static_cast<size_t>(t) * (D / 2) + col / 2);
-      const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.rope_src[which]) + off);
-      float x[8] = {bf16lo_to_f32(u.x), bf16hi_to_f32(u.x), bf16lo_to_f32(u.y), bf16hi_to_f32(u.y),
-                    bf16lo_to_f32(u.z), bf16hi_to_f32(u.z), bf16lo_to_f32(u.w), bf16hi_to_f32(u.w)};
-      rope_rotate_pair(x[0], x[1], c.x, sn.x);
-      rope_rotate_pair(x[2], x[3], c.y, sn.y);
-      rope_rotate_pair(x[4], x[5], c.z, sn.z);
-      rope_rotate_pair(x[6], x[7], c.w, sn.w);
-      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.rope_dst[which]) + off) =
-          make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
-                     pack_bf16x2(x[6], x[7]));
+    for (int i = 0; i < kRopeInFlight; ++i) {
+      const unsigned v = v0 + i * stride;
+      if (v < total) {
+        which[i] = v / per_tensor;
+        e[i] = v - which[i] * per_tensor;  // vector within the tensor
+        const unsigned r = e[i] / VPR, col = (e[i] % VPR) * 8;
+        const unsigned t = (r / p.H) % p.L;  // token
+        const size_t a = static_cast<size_t>(t) * (D / 2) + col / 2;
+        const void* src = which[i] == 0 ? p.rope_src[0]
+                          : which[i] == 1 ? p.rope_src[1]
+                          : which[i] == 2 ? p.rope_src[2]
+                                          : p.rope_src[3];
+        c[i] = *reinterpret_cast<const float4*>(p.rope_cos + a);
+        sn[i] = *reinterpret_cast<const float4*>(p.rope_sin + a);
+        u[i] = reinterpret_cast<const uint4*>(src)[e[i]];
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kRopeInFlight; ++i) {
+      if (v0 + i * stride < total) {
+        float x[8] = {bf16lo_to_f32(u[i].x), bf16hi_to_f32(u[i].x), bf16lo_to_f32(u[i].y),
+                      bf16hi_to_f32(u[i].y), bf16lo_to_f32(u[i].z), bf16hi_to_f32(u[i].z),
+                      bf16lo_to_f32(u[i].w), bf16hi_to_f32(u[i].w)};
+        rope_rotate_pair(x[0], x[1], c[i].x, sn[i].x);
+        rope_rotate_pair(x[2], x[3], c[i].y, sn[i].y);
+        rope_rotate_pair(x[4], x[5], c[i].z, sn[i].z);
+        rope_rotate_pair(x[6], x[7], c[i].w, sn[i].w);
+        void* dst = which[i] == 0 ? p.rope_dst[0]
+                    : which[i] == 1 ? p.rope_dst[1]
+                    : which[i] == 2 ? p.rope_dst[2]
+                                    : p.rope_dst[3];
+        reinterpret_cast<uint4*>(dst)[e[i]] =
+            make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                       pack_bf16x2(x[6], x[7]));
+      }
     }
   }
 }

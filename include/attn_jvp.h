@@ -370,7 +370,8 @@ int attn_jvp_rope(const attn_jvp_shape* shape,
  * to 1024 such calls may be in flight on a device at once. fp32: the
  * rotation pass and then the CUDA-core kernel (two launches).
  *
- * All pointers 16-byte aligned; B * L * H < 2^32 (else ATTN_JVP_ERR_UNSUPPORTED).
+ * All pointers 16-byte aligned; B * L * H * head_dim / 2 < 2^32 (else
+ * ATTN_JVP_ERR_UNSUPPORTED).
  * Returns ATTN_JVP_OK after enqueueing, or an error code with nothing
  * launched. Does not synchronize; a bounded wait that runs out (the grid
  * barrier included) is reported by attn_jvp_sync_status.

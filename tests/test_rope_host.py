@@ -38,3 +38,31 @@ def test_rejects_null_and_misaligned_pointers(lib, i):
     ptrs = list(FAKE)
     ptrs[i] += 4
     assert _rope(lib, s, ptrs) == _abi.ERR_MISALIGNED
+
+
+# attn_jvp_fwd_rope: q k v tq tk tv cos sin, then q' k' tq' tk' o to lse
+FUSED = [0x10000 * (i + 1) for i in range(15)]
+
+
+def _fused(lib, shape, mask, ptrs):
+    return lib.attn_jvp_fwd_rope(ctypes.byref(shape), *ptrs[:8], mask, *ptrs[8:], None)
+
+
+def test_fused_checks_pointers(lib):
+    s = _abi.Shape(1, 64, 2, 64, _abi.DTYPE_BF16, 0.0)
+    m = _abi.Mask(0, 16, 2)  # teacher forcing, 2 chunks of 16: L = 64
+    for i in range(15):
+        ptrs = list(FUSED)
+        ptrs[i] = None
+        assert _fused(lib, s, m, ptrs) == _abi.ERR_INVALID_ARGUMENT
+        ptrs = list(FUSED)
+        ptrs[i] += 8
+        assert _fused(lib, s, m, ptrs) == _abi.ERR_MISALIGNED
+
+
+def test_fused_rejects_more_than_2_32_vectors(lib):
+    # the rotation counts the four tensors' 16-byte vectors in 32 bits:
+    # B L H d / 2 must stay below 2^32
+    m = _abi.Mask(0, 1 << 14, 32)  # L = 2^20
+    at = _abi.Shape(1, 1 << 20, 64, 128, _abi.DTYPE_BF16, 0.0)  # 2^26 rows x 64 = 2^32
+    assert _fused(lib, at, m, FUSED) == _abi.ERR_UNSUPPORTED

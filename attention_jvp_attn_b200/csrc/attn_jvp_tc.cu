@@ -111,11 +111,13 @@ struct TcCfg {
   static constexpr uint32_t TM_TS = 128;
   static constexpr uint32_t TM_P = TM_TS;       // bf16 P over the first half of each warpgroup's tS'
   static constexpr uint32_t TM_U = TM_TS + 32;  // bf16 U over the second half
-  static constexpr uint32_t TM_A = 256;
-  static constexpr uint32_t TM_T = 256 + D;
+  // d = 64: T then A, adjacent, so that one N = 128 group writes [P tV | P V]
+  // from the adjacent (tV, V) tiles of a ring element
+  static constexpr uint32_t TM_A = PAIR ? 256 : 256 + D;
+  static constexpr uint32_t TM_T = PAIR ? 256 + D : 256;
   static constexpr uint32_t TM_COLS = 512;
   static_assert(BYTES <= 232448, "shared memory budget");
-  static_assert(TM_T + D <= TM_COLS, "TMEM budget");
+  static_assert(TM_T + D <= TM_COLS && TM_A + D <= TM_COLS, "TMEM budget");
 };
 
 // Bit mask of the lowest n bits (n clamped to [0, 32]).
@@ -537,6 +539,7 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
     if (mma_cta) {
       const uint32_t idesc_s = idesc_bf16_f32(C::M_MMA, C::BN, 0);
       const uint32_t idesc_v = idesc_bf16_f32(C::M_MMA, D, 1);
+      const uint32_t idesc_v2 = idesc_bf16_f32(C::M_MMA, 2 * D, 1);
       const uint32_t aQ = smem_u32(sQ), aTQ = smem_u32(sTQ), aRing = smem_u32(sRing);
       auto el_addr = [&](uint32_t j) { return aRing + (j % C::NP) * 2 * C::TILE; };
       auto el_ph = [&](uint32_t j) { return (j / C::NP) & 1; };
@@ -617,10 +620,17 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
           p_ph ^= 1;
           AJVP_EV(g, 1);
           tc_fence_after();
-          mma_values_split<C::BN, PAIR>(tmem + C::TM_T, tmem + C::TM_P, aTV, idesc_v, idx > 0);
-          mma_values_split<C::BN, PAIR, 3>(tmem + C::TM_A, tmem + C::TM_P, aV, idesc_v, idx > 0, [&] {
-            rdy_u = test(u_full, u_ph);
-          });
+          if constexpr (PAIR) {
+            mma_values_split<C::BN, PAIR>(tmem + C::TM_T, tmem + C::TM_P, aTV, idesc_v, idx > 0);
+            mma_values_split<C::BN, PAIR, 3>(tmem + C::TM_A, tmem + C::TM_P, aV, idesc_v, idx > 0, [&] {
+              rdy_u = test(u_full, u_ph);
+            });
+          } else {
+            // [T | A] (+)= P [tV | V]: the two 64-column tiles as one N = 128 operand
+            mma_values_split<C::BN, PAIR, 3>(tmem + C::TM_T, tmem + C::TM_P, aTV, idesc_v2, idx > 0, [&] {
+              rdy_u = test(u_full, u_ph);
+            });
+          }
           AJVP_EV(g, 2);
           // D
           if (!rdy_u && !wwait(u_full, u_ph)) break;

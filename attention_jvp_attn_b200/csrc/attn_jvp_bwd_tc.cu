@@ -18,22 +18,20 @@
 //      serves as scratch until launch 3 overwrites it. Padded rows i >= L get
 //      D = 0 and LSE = +inf, so their P is exactly 0.
 //   2. bwd_dkdv_tc_kernel: one CTA per 128 keys of a (batch, head). dK and dV
-//      stay in TMEM while the CTA streams, 64 query rows at a time, the query
-//      tiles whose key-tile schedule lists this key tile (the forward's
-//      schedule, transposed), from separate Q and dO rings:
-//        S^T = K Q^T, dP^T = V dO^T            (SS MMAs, K and V resident,
-//                                               two TMEM buffers of each)
-//        P^T, dS^T in registers (bf16 copies back to TMEM over S^T, dP^T)
+//      stay in TMEM while the CTA streams the 128-row query tiles whose
+//      key-tile schedule lists this key tile (the forward's schedule,
+//      transposed), from separate Q and dO rings:
+//        S^T = K Q^T, dP^T = V dO^T            (SS MMAs, K and V resident)
+//        P^T, dS^T in registers (bf16 copies back to TMEM over dP^T)
 //        dV += P^T dO, dK += dS^T Q            (A operand read from TMEM)
 //   3. bwd_dq_tc_kernel: one CTA per 128 query rows, over the key tiles of the
 //      forward's schedule, from separate K and V rings:
 //        S = Q K^T, dP = dO V^T (two dP buffers), dS in registers,
 //        dQ += dS K                            (A operand read from TMEM)
 //      It forms D_i itself from O and dO, since it overwrites the scratch.
-// Warp roles (320 threads): warps 0-7 two "softmax" warpgroups (each owns half
-// of a tile's columns: 32 of 64 in the dK/dV kernel, 64 of 128 in the dQ
-// kernel), warp 8 TMA producer, warp 9 MMA issuer and TMEM allocator. Every
-// wait is bounded (see ptx.cuh).
+// Warp roles (320 threads): warps 0-7 two "softmax" warpgroups (each owns 64
+// of a tile's 128 columns), warp 8 TMA producer, warp 9 MMA issuer and TMEM
+// allocator. Every wait is bounded (see ptx.cuh).
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -53,7 +51,6 @@ constexpr float kLog2eF = 1.4426950408889634f;
 
 struct BwdTcParams {
   CUtensorMap map_q, map_k, map_v, map_do;  // [B, L, H, d] bf16, boxes of 64 columns x 128 rows
-  CUtensorMap map_q64, map_do64;            // the same for Q and dO, boxes of 64 x 64 rows
   const __nv_bfloat16* o;
   const __nv_bfloat16* dout;
   const float* lse;
@@ -171,43 +168,29 @@ __device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const uint32_
 }
 
 // ---------------------------------------------------------------- dK, dV
-// Query tiles of 64 rows: a stage is a quarter of the 128-key block's
-// operands, so the rings hold several tiles ahead of the MMAs (the loads
-// come from L2 and take a few thousand cycles to land), and TMEM holds two
-// tiles of S^T and dP^T, so the next tile's scores run while the softmax
-// turns the current ones into P^T and dS^T.
-constexpr int kBQ = 64;  // query rows per dK/dV tile
-
+// Query tiles of 128 rows, as in the forward: the score MMAs are N = 128 wide
+// (at N = 64 the tensor core takes about as long for half the work), and TMEM
+// holds one S^T and one dP^T tile beside dV and dK (128 + 128 + 2 d columns).
+// As in the forward, the softmax writes bf16 P^T and dS^T over dP^T (each
+// warpgroup: P^T over the first 32 of its 64 columns, dS^T over the second
+// 32), so S^T is free as soon as the softmax has read it, and S^T_{g+1} runs
+// while the softmax finishes tile g.
 template <int D>
 struct DkdvCfg {
   static constexpr int CH = D / 64;
-  static constexpr int KTILE = kBB * D * 2;           // bytes of a [128 x D] tile (K, V)
-  static constexpr int QTILE = kBQ * D * 2;           // bytes of a [64 x D] tile (Q, dO)
-  static constexpr int QSLOT = QTILE + 1024;          // Q, then LSE log2 e [64] and D [64]
-  static constexpr int NQ = D == 128 ? 5 : 8;         // Q ring slots (released after dK)
-  static constexpr int ND = D == 128 ? 4 : 8;         // dO ring slots (released after dV)
-  static constexpr int DATA = 2 * KTILE + NQ * QSLOT + ND * QTILE;
-  static constexpr int NBAR = 2 * NQ + 2 * ND + 12;
+  static constexpr int TILE = kBB * D * 2;            // bytes of a [128 x D] bf16 tile
+  static constexpr int QSLOT = TILE + 1024;           // Q, then LSE log2 e [128] and D [128]
+  static constexpr int NQ = D == 128 ? 2 : 4;         // Q ring slots (released after dK)
+  static constexpr int ND = D == 128 ? 2 : 4;         // dO ring slots (released after dV)
+  static constexpr int DATA = 2 * TILE + NQ * QSLOT + ND * TILE;
+  static constexpr int NBAR = 2 * NQ + 2 * ND + 10;
   static constexpr int BYTES = 1024 + DATA + NBAR * 8 + 16;
-  // TMEM columns: S^T of tiles 0, 1 (mod 2), dP^T of tiles 0, 1, dV, dK. In a
-  // warpgroup's 32 columns of a buffer, bf16 P^T (dS^T) sits over the first 16.
-  static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 256 + D, TM_COLS = 512;
-  static_assert(QSLOT % 1024 == 0 && QTILE % 1024 == 0, "1024-byte aligned swizzled tiles");
+  // TMEM columns: S^T, dP^T (bf16 P^T and dS^T over it), dV, dK
+  static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_P = TM_DP, TM_DS = TM_DP + 32;
+  static constexpr uint32_t TM_DV = 256, TM_DK = 256 + D, TM_COLS = 512;
+  static_assert(QSLOT % 1024 == 0 && TILE % 1024 == 0, "1024-byte aligned swizzled tiles");
   static_assert(BYTES <= 232448, "shared memory budget");
 };
-
-// Value MMA of the dK/dV kernel: D[tmem] (+)= A[tmem] B, A a bf16 [128 x 64]
-// tile in TMEM in which warpgroup w holds queries [32 w, 32 w + 32) packed in
-// its first 16 columns, B a [64 queries x D] tile read MN-major.
-template <bool Dummy = true>
-__device__ __forceinline__ void mma_values_q64(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem,
-                                               uint32_t idesc, bool accumulate) {
-  const uint64_t db = smem_desc_sw128(b_smem, kBQ * 128, 1024);
-#pragma unroll
-  for (int ks = 0; ks < kBQ / 16; ++ks)
-    umma_ts(d_tmem, a_tmem + 32 * (ks >> 1) + (ks & 1) * 8, db + ((ks * 16 * 128) >> 4), idesc,
-            (accumulate || ks > 0) ? 1u : 0u);
-}
 
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_tc_kernel(const __grid_constant__ BwdTcParams p) {
@@ -216,8 +199,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_tc_kernel(const __gri
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sK = smem;
-  uint8_t* sV = smem + C::KTILE;
-  uint8_t* sQ = smem + 2 * C::KTILE;                 // [NQ] Q slots
+  uint8_t* sV = smem + C::TILE;
+  uint8_t* sQ = smem + 2 * C::TILE;                  // [NQ] Q slots
   uint8_t* sDO = sQ + C::NQ * C::QSLOT;              // [ND] dO slots
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::DATA);
   uint64_t* q_full = bars;                           // [NQ]
@@ -225,12 +208,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_tc_kernel(const __gri
   uint64_t* do_full = bars + 2 * C::NQ;              // [ND]
   uint64_t* do_empty = do_full + C::ND;              // [ND]
   uint64_t* kv_full = do_empty + C::ND;
-  uint64_t* s_full = kv_full + 1;    // [2] S^T of the tile in buffer b
-  uint64_t* dp_full = kv_full + 3;   // [2] dP^T
-  uint64_t* p_full = kv_full + 5;    // [2] P^T (bf16) written
-  uint64_t* ds_full = kv_full + 7;   // [2] dS^T (bf16) written
-  uint64_t* acc_full = kv_full + 9;  // dK, dV complete
-  uint64_t* drain = kv_full + 10;
+  uint64_t* s_full = kv_full + 1;    // S^T of the current tile
+  uint64_t* s_free = kv_full + 2;    // the softmax has read it
+  uint64_t* dp_full = kv_full + 3;   // dP^T
+  uint64_t* p_full = kv_full + 4;    // P^T (bf16) written
+  uint64_t* ds_full = kv_full + 5;   // dS^T (bf16) written
+  uint64_t* acc_full = kv_full + 6;  // dK, dV complete
+  uint64_t* drain = kv_full + 7;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -239,7 +223,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_tc_kernel(const __gri
   const int bh = blockIdx.x / p.n_kt;
   const int kt = blockIdx.x - bh * p.n_kt;
   const int b = bh / p.H, h = bh - b * p.H;
-  const int n_q64 = p.Lp / kBQ;
   MaskSpec mask = p.mask;
   mask.groups = p.groups;
   auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
@@ -256,12 +239,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_tc_kernel(const __gri
       mbar_init(&do_empty[i], 1);
     }
     mbar_init(kv_full, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&dp_full[i], 1);
-      mbar_init(&p_full[i], 8);
-      mbar_init(&ds_full[i], 8);
-    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 8);
+    mbar_init(dp_full, 1);
+    mbar_init(p_full, 8);
+    mbar_init(ds_full, 8);
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -280,14 +262,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_tc_kernel(const __gri
     // ------------------------------------------------------------ producer
     // K and V of the block, then per visited query tile g: Q_g with its LSE
     // and D rows (Q ring), dO_g (dO ring).
-    tma_prefetch_desc(&p.map_q64);
+    tma_prefetch_desc(&p.map_q);
     tma_prefetch_desc(&p.map_k);
     tma_prefetch_desc(&p.map_v);
-    tma_prefetch_desc(&p.map_do64);
+    tma_prefetch_desc(&p.map_do);
     const uint64_t keep = l2_policy_evict_last();   // Q, dO: read by every key block of the head
     const uint64_t once = l2_policy_evict_first();  // K, V: this CTA only
     if (elect_one()) {
-      mbar_arrive_expect_tx(kv_full, 2 * C::KTILE);
+      mbar_arrive_expect_tx(kv_full, 2 * C::TILE);
 #pragma unroll
       for (int c = 0; c < C::CH; ++c) {
         tma_load_4d_hint(sK + c * kBB * 128, &p.map_k, kv_full, c * 64, h, kt * kBB, b, once);
@@ -299,33 +281,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_tc_kernel(const __gri
     const float* d_row = p.scratch + static_cast<size_t>(bh) * p.Lp;
     const float* l_row = p.scratch + total + static_cast<size_t>(bh) * p.Lp;
     ColScan cs;
-    col_scan_start(mask, cs, kt, n_q64, kBQ);
+    col_scan_start(mask, cs, kt, p.n_qt, kBB);
     int qn = 0, dn = 0;  // Q and dO tiles issued
     bool ok = true;
     int qt;
     bool fl;
-    while (col_next(mask, cs, qt, fl, kBQ)) {
+    while (col_next(mask, cs, qt, fl, kBB)) {
       const int g = qn;
       const uint32_t sq = g % C::NQ, sd = g % C::ND;
       if (!wwait(&q_empty[sq], ((g / C::NQ) & 1) ^ 1)) { ok = false; break; }
       uint8_t* qs = sQ + sq * C::QSLOT;
       if (elect_one()) {
-        mbar_arrive_expect_tx(&q_full[sq], C::QTILE + 2 * kBQ * 4);
+        mbar_arrive_expect_tx(&q_full[sq], C::TILE + 2 * kBB * 4);
 #pragma unroll
         for (int c = 0; c < C::CH; ++c)
-          tma_load_4d_hint(qs + c * kBQ * 128, &p.map_q64, &q_full[sq], c * 64, h, qt * kBQ, b, keep);
-        bulk_load(qs + C::QTILE, l_row + qt * kBQ, kBQ * 4, &q_full[sq]);
-        bulk_load(qs + C::QTILE + kBQ * 4, d_row + qt * kBQ, kBQ * 4, &q_full[sq]);
+          tma_load_4d_hint(qs + c * kBB * 128, &p.map_q, &q_full[sq], c * 64, h, qt * kBB, b, keep);
+        bulk_load(qs + C::TILE, l_row + qt * kBB, kBB * 4, &q_full[sq]);
+        bulk_load(qs + C::TILE + kBB * 4, d_row + qt * kBB, kBB * 4, &q_full[sq]);
       }
       __syncwarp();
       qn = g + 1;
       if (!wwait(&do_empty[sd], ((g / C::ND) & 1) ^ 1)) { ok = false; break; }
       if (elect_one()) {
-        mbar_arrive_expect_tx(&do_full[sd], C::QTILE);
+        mbar_arrive_expect_tx(&do_full[sd], C::TILE);
 #pragma unroll
         for (int c = 0; c < C::CH; ++c)
-          tma_load_4d_hint(sDO + sd * C::QTILE + c * kBQ * 128, &p.map_do64, &do_full[sd], c * 64, h,
-                           qt * kBQ, b, keep);
+          tma_load_4d_hint(sDO + sd * C::TILE + c * kBB * 128, &p.map_do, &do_full[sd], c * 64, h,
+                           qt * kBB, b, keep);
       }
       __syncwarp();
       dn = g + 1;
@@ -341,59 +323,62 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_tc_kernel(const __gri
     __syncwarp();
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    // Scores of tile g go to TMEM buffer g % 2. Per tile g: dV_g (after
-    // P^T_g), dK_g (after dS^T_g), then S^T_{g+2} and dP^T_{g+2} into the same
-    // buffer: one thread's tcgen05.mma execute in issue order, so they follow
-    // dV_g's and dK_g's reads of P^T_g and dS^T_g. Meanwhile the softmax
-    // works on tile g+1, whose scores were issued a tile earlier.
-    const uint32_t idesc_s = idesc_bf16_f32(128, kBQ, 0);
+    // Per tile g (all single TMEM buffers):
+    //   C: S^T_{g+1} = K Q_{g+1}^T   once the softmax has read S^T_g (s_free)
+    //   A: dV += P^T_g dO_g          after P^T_g (p_full)
+    //   B: dK += dS^T_g Q_g          after dS^T_g (ds_full)
+    //   E: dP^T_{g+1} = V dO_{g+1}^T over the columns of P^T_g and dS^T_g:
+    //      one thread's tcgen05.mma execute in order, so it follows A and B.
+    // The softmax releases S^T_g before P^T_g is ready, so waiting for s_free
+    // first never delays A and B.
+    const uint32_t idesc_s = idesc_bf16_f32(128, kBB, 0);
     const uint32_t idesc_v = idesc_bf16_f32(128, D, 1);
     const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
     const uint32_t aQ0 = smem_u32(sQ), aD0 = smem_u32(sDO);
     auto q_addr = [&](int g) { return aQ0 + (g % C::NQ) * C::QSLOT; };
-    auto do_addr = [&](int g) { return aD0 + (g % C::ND) * C::QTILE; };
-    // scores of tile j into buffer j % 2
-    auto issue_scores = [&](int j) -> bool {
-      const int bf = j & 1;
+    auto do_addr = [&](int g) { return aD0 + (g % C::ND) * C::TILE; };
+    auto issue_s = [&](int j) -> bool {
       if (!wwait(&q_full[j % C::NQ], (j / C::NQ) & 1)) return false;
       tc_fence_after();
-      mma_scores<D, kBB, kBQ, false>(tmem + C::TM_S + 64 * bf, aK, q_addr(j), idesc_s, false);
-      umma_commit(&s_full[bf]);
+      mma_scores<D, kBB, kBB, false>(tmem + C::TM_S, aK, q_addr(j), idesc_s, false);
+      umma_commit(s_full);
+      return true;
+    };
+    auto issue_dp = [&](int j) -> bool {
       if (!wwait(&do_full[j % C::ND], (j / C::ND) & 1)) return false;
       tc_fence_after();
-      mma_scores<D, kBB, kBQ, false>(tmem + C::TM_DP + 64 * bf, aV, do_addr(j), idesc_s, false);
-      umma_commit(&dp_full[bf]);
+      mma_scores<D, kBB, kBB, false>(tmem + C::TM_DP, aV, do_addr(j), idesc_s, false);
+      umma_commit(dp_full);
       return true;
     };
     ColScan cs;
-    col_scan_start(mask, cs, kt, n_q64, kBQ);
+    col_scan_start(mask, cs, kt, p.n_qt, kBB);
     int qt;
     bool fl;
-    int n_tiles = 0;  // tiles found so far by the scan (the MMA warp runs two ahead)
-    bool ok = true;
-    if (wwait(kv_full, 0)) {
-      for (; n_tiles < 2 && col_next(mask, cs, qt, fl, kBQ); ++n_tiles)
-        if (!issue_scores(n_tiles)) { ok = false; break; }
-    } else {
-      ok = false;
-    }
-    for (int g = 0; ok && g < n_tiles; ++g) {
-      const int bf = g & 1;
-      const uint32_t ph = (g >> 1) & 1;
-      if (!wwait(&p_full[bf], ph)) break;
+    bool ok = wwait(kv_full, 0);
+    bool has = ok && col_next(mask, cs, qt, fl, kBB);
+    if (has) ok = issue_s(0) && issue_dp(0);
+    for (int g = 0; ok && has; ++g) {
+      const uint32_t ph = g & 1;
+      const bool next = col_next(mask, cs, qt, fl, kBB);
+      // C
+      if (next && (!wwait(s_free, ph) || !issue_s(g + 1))) break;
+      // A
+      if (!wwait(p_full, ph)) break;
       tc_fence_after();
-      mma_values_q64(tmem + C::TM_DV, tmem + C::TM_S + 64 * bf, do_addr(g), idesc_v, g > 0);
+      mma_values_split<kBB, false>(tmem + C::TM_DV, tmem + C::TM_P, do_addr(g), idesc_v, g > 0);
       umma_commit(&do_empty[g % C::ND]);
-      if (!wwait(&ds_full[bf], ph)) break;
+      // B
+      if (!wwait(ds_full, ph)) break;
       tc_fence_after();
-      mma_values_q64(tmem + C::TM_DK, tmem + C::TM_DP + 64 * bf, q_addr(g), idesc_v, g > 0);
+      mma_values_split<kBB, false>(tmem + C::TM_DK, tmem + C::TM_DS, q_addr(g), idesc_v, g > 0);
       umma_commit(&q_empty[g % C::NQ]);
-      if (col_next(mask, cs, qt, fl, kBQ)) {
-        if (!issue_scores(n_tiles)) break;
-        ++n_tiles;
-      } else if (g == n_tiles - 1) {
+      if (!next) {
         umma_commit(acc_full);
+        break;
       }
+      // E
+      if (!issue_dp(g + 1)) break;
     }
     // Every MMA issued so far completes before TMEM is released.
     umma_commit(drain);
@@ -402,57 +387,61 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_tc_kernel(const __gri
   } else {
     // ------------------------------------------------------------ softmax + epilogue
     // Thread (wg, sub, lane) owns key row 32 sub + lane (its TMEM lane) and the
-    // query columns [32 wg, 32 wg + 32) of every 64-row query tile.
+    // query columns [64 wg, 64 wg + 64) of every 128-row query tile.
     const int wg = warp >> 2, sub = warp & 3;
     const int row = sub * 32 + lane;
     const int key = kt * kBB + row;
     const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
+    const uint32_t tS = tmem + lane_off + C::TM_S + 64 * wg;
+    const uint32_t tDP = tmem + lane_off + C::TM_DP + 64 * wg;
     const uint32_t tDV = tmem + lane_off + C::TM_DV + (D / 2) * wg;
     const uint32_t tDK = tmem + lane_off + C::TM_DK + (D / 2) * wg;
     const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
     ColScan cs;
-    col_scan_start(mask, cs, kt, n_q64, kBQ);
+    col_scan_start(mask, cs, kt, p.n_qt, kBB);
     int g = 0;
     bool ok = true;
     int qt;
     bool fl;
-    while (col_next(mask, cs, qt, fl, kBQ)) {
-      const int bf = g & 1;
-      const uint32_t ph = (g >> 1) & 1;
-      const uint32_t tS = tmem + lane_off + C::TM_S + 64 * bf + 32 * wg;
-      const uint32_t tDP = tmem + lane_off + C::TM_DP + 64 * bf + 32 * wg;
+    while (col_next(mask, cs, qt, fl, kBB)) {
+      const uint32_t ph = g & 1;
       const float* lse2 =
-          reinterpret_cast<const float*>(sQ + (g % C::NQ) * C::QSLOT + C::QTILE) + 32 * wg;
-      const float* dd = lse2 + kBQ;
+          reinterpret_cast<const float*>(sQ + (g % C::NQ) * C::QSLOT + C::TILE) + 64 * wg;
+      const float* dd = lse2 + kBB;
       // the tile's LSE and D are read from shared memory: observe its copies
       if (!wwait(&q_full[g % C::NQ], (g / C::NQ) & 1)) { ok = false; break; }
-      if (!wwait(&s_full[bf], ph)) { ok = false; break; }
+      if (!wwait(s_full, ph)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sr[32];
-      tmem_ld32(tS, sr);
+      uint32_t sr[64];
+      tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       tmem_wait_ld();
+      // S^T_g is in registers: the MMA warp may write S^T_{g+1}
+      tc_fence_before();
+      __syncwarp();
+      mbar_arrive_if(s_free, lane == 0);
       if (!fl) {
         // Admissible query columns of this key, row group by row group.
-        uint32_t m = 0;
-        int i = qt * kBQ + 32 * wg;
+        uint32_t m[2] = {0u, 0u};
+        int i = qt * kBB + 64 * wg;
         RowRange rr = row_range(mask, i);
         int nxt = next_group_start(mask, i);
 #pragma unroll 1
-        for (int c = 0; c < 32; ++c, ++i) {
+        for (int c = 0; c < 64; ++c, ++i) {
           if (i >= nxt) {
             rr = row_range(mask, i);
             nxt = next_group_start(mask, i);
           }
-          m |= (row_allows(rr, key) ? 1u : 0u) << c;
+          m[c >> 5] |= (row_allows(rr, key) ? 1u : 0u) << (c & 31);
         }
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (!((m >> j) & 1u)) sr[j] = __float_as_uint(-INFINITY);
+        for (int j = 0; j < 64; ++j)
+          if (!((m[j >> 5] >> (j & 31)) & 1u)) sr[j] = __float_as_uint(-INFINITY);
       }
       // P^T = 2^(S^T s log2 e - LSE_i log2 e): 0 where masked or past L
-      uint32_t pk[16];
+      uint32_t pk[32];
 #pragma unroll
-      for (int j = 0; j < 32; j += 4) {
+      for (int j = 0; j < 64; j += 4) {
         const float4 l4 = *reinterpret_cast<const float4*>(lse2 + j);
         const float2 x01 = __ffma2_rn(make_float2(__uint_as_float(sr[j]), __uint_as_float(sr[j + 1])),
                                       sc2, make_float2(-l4.x, -l4.y));
@@ -467,31 +456,45 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_tc_kernel(const __gri
         pk[j / 2] = pack_bf16x2(p0, p1);
         pk[j / 2 + 1] = pack_bf16x2(p2, p3);
       }
-      tmem_st16(tS, pk);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      mbar_arrive_if(&p_full[bf], lane == 0);
-      // dS^T = P^T (dP^T - D_i) on pairs of floats, over the first half of
-      // this warpgroup's dP^T columns
-      if (!wwait(&dp_full[bf], ph)) { ok = false; break; }
+      // dS^T = P^T (dP^T - D_i) on pairs of floats, in two halves of 32
+      // queries: P^T goes over the first half of this warpgroup's dP^T columns
+      // once it is read, dS^T over the second.
+      if (!wwait(dp_full, ph)) { ok = false; break; }
       tc_fence_after();
-      uint32_t v[32];
-      tmem_ld32(tDP, v);
-      tmem_wait_ld();
+      uint32_t dk[32];
+      auto ds_half = [&](int hq, const uint32_t (&v)[32]) {
 #pragma unroll
-      for (int j = 0; j < 32; j += 2) {
-        const float2 d2 = *reinterpret_cast<const float2*>(dd + j);
-        const float2 ds = __fmul2_rn(make_float2(__uint_as_float(sr[j]), __uint_as_float(sr[j + 1])),
-                                     __fadd2_rn(make_float2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])),
-                                                make_float2(-d2.x, -d2.y)));
-        pk[j / 2] = pack_bf16x2(ds.x, ds.y);
+        for (int j = 0; j < 32; j += 2) {
+          const float2 d2 = *reinterpret_cast<const float2*>(dd + 32 * hq + j);
+          const float2 ds = __fmul2_rn(
+              make_float2(__uint_as_float(sr[32 * hq + j]), __uint_as_float(sr[32 * hq + j + 1])),
+              __fadd2_rn(make_float2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])),
+                         make_float2(-d2.x, -d2.y)));
+          dk[16 * hq + j / 2] = pack_bf16x2(ds.x, ds.y);
+        }
+      };
+      {
+        uint32_t v[32];
+        tmem_ld32(tDP, v);
+        tmem_wait_ld();
+        ds_half(0, v);
       }
-      tmem_st16(tDP, pk);
+      tmem_st32(tDP, pk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      mbar_arrive_if(&ds_full[bf], lane == 0);
+      mbar_arrive_if(p_full, lane == 0);
+      {
+        uint32_t v[32];
+        tmem_ld32(tDP + 32, v);
+        tmem_wait_ld();
+        ds_half(1, v);
+      }
+      tmem_st32(tDP + 32, dk);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      mbar_arrive_if(ds_full, lane == 0);
       ++g;
     }
     // ---------------- epilogue: dV, s dK of this key (zero if no query sees it)
@@ -919,9 +922,7 @@ int bwd_tc_launch(const BwdTcArgs& a, cudaStream_t stream) {
   if (!encode_bf16_rows_map(&p.map_q, a.q, a.B, a.L, a.H, a.d, kBB) ||
       !encode_bf16_rows_map(&p.map_k, a.k, a.B, a.L, a.H, a.d, kBB) ||
       !encode_bf16_rows_map(&p.map_v, a.v, a.B, a.L, a.H, a.d, kBB) ||
-      !encode_bf16_rows_map(&p.map_do, a.dout, a.B, a.L, a.H, a.d, kBB) ||
-      !encode_bf16_rows_map(&p.map_q64, a.q, a.B, a.L, a.H, a.d, kBQ) ||
-      !encode_bf16_rows_map(&p.map_do64, a.dout, a.B, a.L, a.H, a.d, kBQ))
+      !encode_bf16_rows_map(&p.map_do, a.dout, a.B, a.L, a.H, a.d, kBB))
     return ATTN_JVP_ERR_CUDA;
   p.o = static_cast<const __nv_bfloat16*>(a.o);
   p.dout = static_cast<const __nv_bfloat16*>(a.dout);

@@ -22,7 +22,8 @@ from .inputs import BLOCK_CAUSAL, TEACHER_FORCING  # noqa: F401
 
 __all__ = ["attn_jvp", "attn_jvp_groups", "attn_jvp_bwd", "attn_jvp_bwd_groups", "rope",
            "attn_jvp_rope", "attn_jvp_host", "sync_status", "unmasked_pairs", "schedule_tiles",
-           "host_staging_bytes", "AttnJvpError", "TEACHER_FORCING", "BLOCK_CAUSAL"]
+           "key_tile_query_bounds", "host_staging_bytes", "AttnJvpError", "TEACHER_FORCING",
+           "BLOCK_CAUSAL"]
 
 _DT = {torch.bfloat16: _abi.DTYPE_BF16, torch.float32: _abi.DTYPE_F32}
 
@@ -279,6 +280,18 @@ def schedule_tiles(mode: int, chunk_tokens: int, n_chunks: int, L: int, block_m:
     full = (ctypes.c_uint8 * max(n, 1))()
     lib.attn_jvp_schedule_tiles(m, L, block_m, block_n, q_tile, tiles, full, n)
     return list(tiles[:n]), list(full[:n])
+
+
+def key_tile_query_bounds(mode: int, chunk_tokens: int, n_chunks: int, L: int, block_m: int,
+                          block_n: int, k_tile: int) -> Tuple[int, int]:
+    """Query tiles [lo, hi] the backward scans for one key tile."""
+    lo, hi = ctypes.c_int32(), ctypes.c_int32()
+    r = _abi.load().attn_jvp_key_tile_query_bounds(_mask(mode, chunk_tokens, n_chunks), L, block_m,
+                                                   block_n, k_tile, ctypes.byref(lo),
+                                                   ctypes.byref(hi))
+    if r != 0:
+        raise ValueError("bad bounds arguments")
+    return lo.value, hi.value
 
 
 def default_scale(d: int) -> float:

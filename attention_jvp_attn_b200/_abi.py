@@ -85,6 +85,10 @@ def load(path: str = None) -> ctypes.CDLL:
                                                 ctypes.POINTER(ctypes.c_int32),
                                                 ctypes.POINTER(ctypes.c_uint8), ctypes.c_int32]
         lib.attn_jvp_schedule_tiles.restype = ctypes.c_int32
+        lib.attn_jvp_key_tile_query_bounds.argtypes = [
+            Mask, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+            ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]
+        lib.attn_jvp_key_tile_query_bounds.restype = ctypes.c_int32
         lib.attn_jvp_fwd_noalloc.argtypes = [ctypes.POINTER(Shape), vp, vp, vp, vp, vp, vp,
                                              Mask, vp, vp, vp, vp]
         lib.attn_jvp_fwd_noalloc.restype = ctypes.c_int

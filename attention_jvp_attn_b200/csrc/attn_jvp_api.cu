@@ -764,6 +764,20 @@ int32_t attn_jvp_schedule_tiles(attn_jvp_mask mask, int64_t L, int32_t block_m, 
   return n;
 }
 
+int32_t attn_jvp_key_tile_query_bounds(attn_jvp_mask mask, int64_t L, int32_t block_m,
+                                       int32_t block_n, int32_t k_tile, int32_t* lo, int32_t* hi) {
+  int64_t Lx = 0;
+  if (validate_mask(mask, &Lx) != ATTN_JVP_OK || Lx != L) return -1;
+  if (block_m < 1 || block_n < 1 || k_tile < 0 || !lo || !hi) return -1;
+  if (int64_t(k_tile) * block_n >= L) return -1;
+  const int n_qt = static_cast<int>((L + block_m - 1) / block_m);
+  int a = 0, b = 0;
+  ajvp::key_tile_query_bounds(mask_spec(mask, L), k_tile, block_n, n_qt, block_m, a, b);
+  *lo = a;
+  *hi = b;
+  return 0;
+}
+
 int32_t attn_jvp_version(void) { return 100; }
 
 int attn_jvp_debug_wait(int64_t limit_ns, int32_t stall_tile) {

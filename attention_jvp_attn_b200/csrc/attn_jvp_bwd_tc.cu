@@ -129,34 +129,13 @@ __device__ __forceinline__ void col_scan_load(const MaskSpec& m, ColScan& cs, in
   cs.full = __ballot_sync(0xffffffffu, f);
 }
 
-// Query tiles [lo, hi] outside which no row can see key tile kt: exact for
-// the closed-form masks (teacher forcing: clean keys are seen from their
-// chunk's clean rows on, noisy keys only by their own chunk's noisy rows;
-// block causal: from the key's chunk on), every tile for a group table. The
-// scan then skips the tiles before lo and stops after hi instead of testing
-// every query tile of the sequence (tens of microseconds per CTA otherwise).
-__device__ __forceinline__ void col_bounds(const MaskSpec& m, int kt, int n_qt, int bq, int& lo,
-                                           int& hi) {
-  lo = 0;
-  hi = n_qt - 1;
-  const int k0 = kt * kBB;
-  if (m.mode == kModeGroups || k0 >= m.L) return;
-  const int c = m.c;
-  const int nc = m.n * c;
-  if (m.mode == kModeTeacherForcing && k0 >= nc) {
-    const int k1 = min(k0 + kBB, m.L) - 1;
-    const int i0 = (k0 - nc) / c, i1 = (k1 - nc) / c;
-    lo = (nc + i0 * c) / bq;
-    hi = min(n_qt - 1, (nc + i1 * c + c - 1) / bq);
-    return;
-  }
-  lo = ((k0 / c) * c) / bq;
-}
-
 __device__ __forceinline__ void col_scan_start(const MaskSpec& m, ColScan& cs, int kt, int n_qt,
                                                int bq) {
+  // Only the query tiles the mask can admit for this key tile: without the
+  // bounds every warp scanned all query tiles of the sequence (tens of
+  // microseconds per CTA).
   int lo, hi;
-  col_bounds(m, kt, n_qt, bq, lo, hi);
+  key_tile_query_bounds(m, kt, kBB, n_qt, bq, lo, hi);
   cs.kt = kt;
   cs.n_qt = hi + 1;
   cs.base = lo;

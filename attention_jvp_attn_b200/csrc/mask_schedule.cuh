@@ -205,4 +205,28 @@ AJVP_HD TileSched make_tile_sched(const MaskSpec& m, int q_tile, int bm, int bn)
   return s;
 }
 
+// Query tiles [lo, hi] (tiles of bq rows, n_qt of them) outside which no row
+// can see key tile kt (tiles of bk keys): exact for the closed-form masks
+// (teacher forcing: clean keys are seen from their chunk's clean rows on,
+// noisy keys only by their own chunk's noisy rows; block causal: from the
+// key's chunk on), every tile for a group table or a tile past L.
+AJVP_HD void key_tile_query_bounds(const MaskSpec& m, int kt, int bk, int n_qt, int bq, int& lo,
+                                   int& hi) {
+  lo = 0;
+  hi = n_qt - 1;
+  const int k0 = kt * bk;
+  if (m.mode == kModeGroups || k0 >= m.L) return;
+  const int c = m.c;
+  const int nc = m.n * c;
+  if (m.mode == kModeTeacherForcing && k0 >= nc) {
+    const int k1 = (k0 + bk < m.L ? k0 + bk : m.L) - 1;  // last key of the tile
+    const int i0 = (k0 - nc) / c, i1 = (k1 - nc) / c;
+    lo = (nc + i0 * c) / bq;
+    const int h = (nc + i1 * c + c - 1) / bq;
+    hi = h < n_qt - 1 ? h : n_qt - 1;
+    return;
+  }
+  lo = ((k0 / c) * c) / bq;
+}
+
 }  // namespace ajvp

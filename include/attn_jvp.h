@@ -422,6 +422,23 @@ int32_t attn_jvp_schedule_tiles_groups(const attn_jvp_group* groups, int32_t n_g
                                        int32_t* tiles, uint8_t* full, int32_t cap);
 
 /*
+ * attn_jvp_key_tile_query_bounds - the range of query tiles [*lo, *hi] that
+ * the backward's dK/dV kernel scans for key tile k_tile (the transpose of
+ * the schedule above: the query tiles whose schedule lists the key tile all
+ * lie in the range). Exact for the closed-form masks (teacher forcing: clean
+ * keys are seen from their chunk's clean rows on, noisy keys only by their
+ * own chunk's noisy rows; block causal: from the key's chunk on).
+ *
+ *   mask, L       mask and sequence length (validated as for attn_jvp_fwd)
+ *   block_m/_n    query / key tile sizes
+ *   k_tile        key tile index, 0 <= k_tile < ceil(L / block_n)
+ *
+ * Returns 0, or -1 on a bad argument (nothing written).
+ */
+int32_t attn_jvp_key_tile_query_bounds(attn_jvp_mask mask, int64_t L, int32_t block_m,
+                                       int32_t block_n, int32_t k_tile, int32_t* lo, int32_t* hi);
+
+/*
  * attn_jvp_debug_wait - TEST ONLY: drives the bf16 forward kernels' bounded
  * waits to run out without a device fault (a wait on a barrier that nothing
  * completes), so that the timeout path can be tested. Not part of the

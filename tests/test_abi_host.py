@@ -183,3 +183,33 @@ def test_debug_wait_settings_are_checked(lib):
     assert lib.attn_jvp_debug_wait(61 * 10**9, -1) == _abi.ERR_INVALID_ARGUMENT
     assert lib.attn_jvp_debug_wait(2_000_000, 3) == _abi.OK
     assert lib.attn_jvp_debug_wait(0, -1) == _abi.OK
+
+
+@pytest.mark.parametrize("mode", [TF, BC])
+@pytest.mark.parametrize("c,n", [(1, 1), (1, 7), (5, 4), (24, 5), (100, 3), (128, 2), (130, 3),
+                                 (150, 3), (200, 2), (1560, 2)])
+@pytest.mark.parametrize("bm,bn", [(128, 128), (64, 128), (32, 32)])
+def test_key_tile_query_bounds_cover_the_explicit_mask(lib, mode, c, n, bm, bn):
+    """The backward's dK/dV kernel scans only the query tiles in these bounds
+    for a key tile: every query tile with an admissible pair in the key tile
+    (from the oracle's explicit mask) must lie inside them, and for these
+    closed-form masks the lower bound is the first such tile."""
+    L = orc.seq_len(mode, c, n)
+    M = orc.mask_matrix(mode, c, n)
+    n_q = -(-L // bm)
+    for kt in range(-(-L // bn)):
+        lo, hi = aj.key_tile_query_bounds(mode, c, n, L, bm, bn, kt)
+        cols = M[:, kt * bn:min(L, (kt + 1) * bn)]
+        seen = [qt for qt in range(n_q) if cols[qt * bm:min(L, (qt + 1) * bm)].any()]
+        assert 0 <= lo <= hi < n_q, (kt, lo, hi)
+        if seen:
+            assert lo == seen[0] and seen[-1] <= hi, (kt, lo, hi, seen[0], seen[-1])
+
+
+def test_key_tile_query_bounds_rejects_bad_arguments(lib):
+    with pytest.raises(ValueError):
+        aj.key_tile_query_bounds(TF, 16, 2, 64, 128, 128, 1)  # key tile past L
+    with pytest.raises(ValueError):
+        aj.key_tile_query_bounds(TF, 16, 2, 65, 128, 128, 0)  # L does not match the mask
+    with pytest.raises(ValueError):
+        aj.key_tile_query_bounds(TF, 16, 2, 64, 0, 128, 0)

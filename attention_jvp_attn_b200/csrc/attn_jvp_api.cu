@@ -384,8 +384,11 @@ int launch_f32(const attn_jvp_shape* s, const void* q, const void* k, const void
 
 int64_t round256(int64_t x) { return (x + 255) & ~int64_t(255); }
 
-// attn_jvp_fwd_host: heads in up to kHostChunks chunks, two staging slots.
-constexpr int64_t kHostChunks = 4;
+// attn_jvp_fwd_host: heads in up to kHostChunks chunks (one head per chunk
+// when H <= kHostChunks), two staging slots. Small chunks keep the part that
+// cannot overlap (the first chunk's copy in, the last chunk's kernel and copy
+// out) short: the copies in are the bulk of the call.
+constexpr int64_t kHostChunks = 16;
 
 // Copy streams and events of attn_jvp_fwd_host, created once per device and
 // kept (like the status word): a call creates nothing.

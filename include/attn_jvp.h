@@ -167,7 +167,8 @@ int attn_jvp_fwd_groups(const attn_jvp_shape* shape,
  * the copies to run at full speed (and to overlap with the kernel); pageable
  * memory also works.
  *
- * The heads go in up to 4 chunks through two staging slots: the copies in
+ * The heads go in up to 16 chunks (one head per chunk when H <= 16) through
+ * two staging slots: the copies in
  * of chunk c+1 and the copies out of chunk c-1 run on two copy streams while
  * the kernel of chunk c runs on `stream`, ordered by events. The copy
  * streams and events are created on the first call on a device and kept
@@ -191,7 +192,7 @@ int attn_jvp_fwd_host(const attn_jvp_shape* shape,
                       void* d_buf, void* stream);
 
 /* Bytes of device staging attn_jvp_fwd_host needs for `shape` (0 on a bad shape):
- * two slots of one chunk of heads (8 tensors and the LSE of ceil(H / 4) heads,
+ * two slots of one chunk of heads (8 tensors and the LSE of ceil(H / 16) heads,
  * each piece rounded up to 256 bytes), or one slot of the whole problem when H = 1. */
 int64_t attn_jvp_host_staging_bytes(const attn_jvp_shape* shape);
 

@@ -162,13 +162,16 @@ def _round256(x):
 
 
 def test_staging_bytes(lib):
-    # heads go in up to 4 chunks through two staging slots, each holding the
+    # heads go in up to 16 chunks through two staging slots, each holding the
     # 8 tensors and the LSE of one chunk (256-byte aligned pieces)
     s = _abi.Shape(2, 128, 3, 64, 0, 0.0)  # 3 chunks of 1 head
     slot = 8 * _round256(2 * 128 * 1 * 64 * 2) + _round256(2 * 1 * 128 * 4)
     assert lib.attn_jvp_host_staging_bytes(ctypes.byref(s)) == 2 * slot
-    s = _abi.Shape(1, 100, 12, 128, 1, 0.0)  # fp32, 4 chunks of 3 heads
-    slot = 8 * _round256(100 * 3 * 128 * 4) + _round256(3 * 100 * 4)
+    s = _abi.Shape(1, 100, 12, 128, 1, 0.0)  # fp32, 12 chunks of 1 head
+    slot = 8 * _round256(100 * 1 * 128 * 4) + _round256(1 * 100 * 4)
+    assert lib.attn_jvp_host_staging_bytes(ctypes.byref(s)) == 2 * slot
+    s = _abi.Shape(1, 100, 40, 64, 0, 0.0)  # 14 chunks of 3 heads (the last one of 1)
+    slot = 8 * _round256(100 * 3 * 64 * 2) + _round256(3 * 100 * 4)
     assert lib.attn_jvp_host_staging_bytes(ctypes.byref(s)) == 2 * slot
     s = _abi.Shape(1, 100, 1, 64, 0, 0.0)  # one head: one slot of the whole problem
     assert lib.attn_jvp_host_staging_bytes(ctypes.byref(s)) == \

@@ -14,8 +14,10 @@
 //         P and U (bf16) written back over tS' (each warpgroup's 64 columns:
 //         32 of P, then 32 of U), which frees the S columns for S_{j+1}
 //         while the softmax of tile j is still running
-//   MMA   A += P V_j                           (TMEM cols [256,256+d))
-//   MMA   T += U V_j + P tV_j                  (TMEM cols [256+d,256+2d))
+//   MMA   A += P V_j                           (d = 128: TMEM cols [256,384))
+//   MMA   T += U V_j + P tV_j                  (d = 128: TMEM cols [384,512))
+//         (d = 64: T at [256,320) and A at [320,384), so that P tV and P V
+//         are one N = 128 MMA group over the adjacent tV and V tiles)
 //   end   O = A/l, mu = D/l, tO = T/l - mu O, LSE = (m + log2 l) ln 2
 // which is tO = sum_j P_ij (tS_ij - mu_i) v_j + sum_j P_ij tv_j with
 // tS = s (tQ K^T + Q tK^T), i.e. tP V + P tV, tP = P (tS - rowsum(P tS)).
@@ -510,7 +512,7 @@ __global__ void __launch_bounds__(kTcThreads) attn_jvp_tc_kernel(const __grid_co
     // Per key tile g, with ring elements KK_j = (K_j, tK_j) and VV_j = (tV_j, V_j):
     //   C: S_{g+1} = Q K_{g+1}^T        once the softmax has read S_g (s_free)
     //   A: T (+)= P_g tV_g              after P_g (p_full)
-    //   B: A (+)= P_g V_g
+    //   B: A (+)= P_g V_g               (d = 64: A and B as one N = 128 group)
     //   D: T += U_g V_g                 after U_g (u_full)
     //   E: tS'_{g+1} = tQ K_{g+1}^T + Q tK_{g+1}^T
     // Within an item C goes first, waiting for s_free if need be: the softmax
